@@ -1,0 +1,1 @@
+"""CPU reference oracle (test infrastructure only; never imported by the product path)."""

@@ -318,7 +318,7 @@ def _coarse_block(idx, b, h, j, L, tok0, unit):
     w = np.diff(off).astype(np.float64)
     u = stream_uniforms(cfg["seed"], unit, j, 1, CC)
     picks = kmeanspp_pick(F, CC, u, w=w)
-    ca, ccent, _ = lloyd(F, F[picks], cfg["iters"], dtype, w=w)
+    ca, ccent, chist = lloyd(F, F[picks], cfg["iters"], dtype, w=w)
     # coarse centroids: means of the member tokens' keys and values
     ids = idx["perm"][b, h, tok0:tok0 + L]                      # token id by store position
     tok_coarse = ca[idx["assign"][b, h, ids] - s0]
@@ -357,7 +357,7 @@ def _coarse_block(idx, b, h, j, L, tok0, unit):
     idx["Vcc"][b, h, t0:t0 + CC] = Vcc
     idx["coff"][b, h, t0:t0 + CC] = s0 + np.concatenate([[0], np.cumsum(ccnt)[:-1]])
     idx["coff"][b, h, t0 + CC:t0 + CC_blk] = s0 + C
-    return {"coarse_assign": ca, "fine_order": fo}
+    return {"coarse_assign": ca, "fine_order": fo, "hist": chist, "points": F, "picks": picks}
 
 
 def _block_init(idx, b, h, j, X, L_old, init_mode, unit, init_given):
@@ -421,7 +421,9 @@ def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None):
             for h in range(H):
                 for j in range(nb):
                     s, e = j * Lb, min(n, (j + 1) * Lb)
-                    _coarse_block(idx, b, h, j, e - s, s, b * H + h)
+                    ch = _coarse_block(idx, b, h, j, e - s, s, b * H + h)
+                    if record is not None:
+                        record[(b, h, j, "coarse")] = ch
         _finish_offsets(idx)
     return idx
 
@@ -521,13 +523,14 @@ def block_tokens_in_order(idx, b, h, j, n_upto):
     return idx["Kp"][b, h, inv], idx["Vp"][b, h, inv]
 
 
-def cluster_update(idx, K_new, V_new):
+def cluster_update(idx, K_new, V_new, record=None):
     """Append generated tokens; re-cluster the blocks holding tail tokens on a trigger.
 
     The trigger (R13): the tail (tokens not yet clustered) holds at least
     ``update_interval`` tokens, or it reaches the end of a block.  Each block
     holding tail tokens is re-clustered over all its tokens with the warm start
-    of R14.  Returns True if a trigger fired.
+    of R14.  Returns True if a trigger fired.  ``record`` (optional list)
+    receives (b, h, j, keys, init, Lloyd history) per re-clustered block.
     """
     cfg = idx["cfg"]
     B, H = cfg["B"], cfg["Hkv"]
@@ -554,7 +557,9 @@ def cluster_update(idx, K_new, V_new):
                 L_old = max(0, min(nc, e) - s)
                 Xk, Xv = block_tokens_in_order(idx, b, h, j, e)
                 ini = _block_init(idx, b, h, j, Xk, L_old, "warm", unit, None)
-                _cluster_block(idx, b, h, j, Xk, Xv, ini)
+                hist = _cluster_block(idx, b, h, j, Xk, Xv, ini)
+                if record is not None:
+                    record.append((b, h, j, Xk, ini, hist))
                 if cfg.get("levels", 1) == 2:
                     _coarse_block(idx, b, h, j, e - s, s, unit)
     idx["n_clustered"] = n1

@@ -1,0 +1,118 @@
+"""Decode parity: the CUDA decode (through the C ABI) against the fp64 oracle.
+
+The index is built by the oracle and uploaded with mp_index_import, so that
+decode parity is checked independently of clustering parity.  Outputs are
+compared element by element (max-abs 2e-2 for bf16 inputs, 1e-4 for fp32);
+selected sets must match exactly unless a score tie within 1e-5 decides them.
+"""
+import numpy as np
+import pytest
+import torch
+
+import helpers as H
+from clustered_sparse_decode_b200 import MultipoleIndex, synth
+from oracle import multipole as mp
+
+pytestmark = pytest.mark.gpu
+
+
+def run_decode(o, oidx, Q, budget, coarse_budget=0, no_approx=False, n_split=0, scale=None):
+    gidx = MultipoleIndex(H.gcfg(o))
+    H.upload_index(gidx, oidx)
+    B, Hkv = o["B"], o["Hkv"]
+    mask = torch.zeros((B, Hkv, gidx.slots), dtype=torch.uint8, device="cuda")
+    scores = torch.empty((B, Hkv, gidx.slots), dtype=torch.float32, device="cuda")
+    cmask = cscores = None
+    if o["levels"] == 2:
+        cmask = torch.zeros((B, Hkv, gidx.coarse_slots), dtype=torch.uint8, device="cuda")
+        cscores = torch.empty((B, Hkv, gidx.coarse_slots), dtype=torch.float32, device="cuda")
+    Qd = H.tdev(Q, o["dtype"])
+    O = gidx.decode(Qd, budget, coarse_budget=coarse_budget, no_approx=no_approx, n_split=n_split,
+                    scale=0.0 if scale is None else scale, sel_mask=mask, scores=scores,
+                    coarse_sel_mask=cmask, coarse_scores=cscores)
+    torch.cuda.synchronize()
+    assert gidx.check_device_error() == 0
+    info = {}
+    O_ref = mp.decode(oidx, Q, budget, coarse_budget=coarse_budget if coarse_budget > 0 else None,
+                      flags=mp.NO_APPROX if no_approx else 0, scale=scale, info=info)
+    skipped = H.compare_decode(o, H.to_np(O), O_ref, info, mask.cpu().numpy(), scores.cpu().numpy(),
+                               levels=o["levels"], gpu_cmask=None if cmask is None else cmask.cpu().numpy())
+    return skipped, H.to_np(O), O_ref
+
+
+GEOMS = {
+    # name: (oracle cfg kwargs, tokens)
+    "f32_d64_g4": (dict(B=1, Hkv=1, Hq=4, d=64, n_max=2048, L_blk=2048, dtype="f32"), 2048),
+    "bf16_d128_g4_ragged": (dict(B=2, Hkv=2, Hq=8, d=128, n_max=5000, L_blk=2048), 4999),
+    "bf16_d128_g1": (dict(B=1, Hkv=3, Hq=3, d=128, n_max=3000, L_blk=1024), 3000),
+    "bf16_d64_g2": (dict(B=2, Hkv=2, Hq=4, d=64, n_max=2500, L_blk=1024), 2400),
+    "bf16_d128_g8": (dict(B=1, Hkv=2, Hq=16, d=128, n_max=2048, L_blk=2048), 2048),
+    "f32_d128_g8": (dict(B=1, Hkv=1, Hq=8, d=128, n_max=1500, L_blk=1024, dtype="f32"), 1500),
+}
+
+
+@pytest.mark.parametrize("geom", list(GEOMS))
+@pytest.mark.parametrize("budget", [0, 1, 100, 100000])
+@pytest.mark.parametrize("no_approx", [False, True])
+def test_decode_matches_oracle(geom, budget, no_approx):
+    kw, n = GEOMS[geom]
+    o = H.ocfg(**kw)
+    K, V, lab = H.cache_for(o, n, comps=48, seed=11)
+    oidx = H.component_index(o, K, V, lab, n)           # 48 components into up to 128 slots: empty clusters
+    Q = synth.make_queries(1, o["B"], o["Hq"], o["d"], o["dtype"], seed=5)[0]
+    skipped, _, _ = run_decode(o, oidx, Q, budget, no_approx=no_approx)
+    assert skipped <= max(1, o["B"] * o["Hkv"] // 4)
+
+
+@pytest.mark.parametrize("n_split", [1, 3, 17, 64])
+def test_split_count_does_not_change_the_result(n_split):
+    o = H.ocfg(B=2, Hkv=2, Hq=8, d=128, n_max=4096, L_blk=2048)
+    K, V, lab = H.cache_for(o, 4096, comps=128, seed=3)
+    oidx = H.component_index(o, K, V, lab, 4096)
+    Q = synth.make_queries(1, 2, 8, 128, "bf16", seed=8)[0]
+    _, O1, ref = run_decode(o, oidx, Q, 700, n_split=n_split)
+    _, O2, _ = run_decode(o, oidx, Q, 700, n_split=1)
+    assert np.abs(O1 - O2).max() <= 4e-3
+
+
+def test_kmeans_index_and_tail_tokens():
+    """An oracle k-means index with an unclustered tail (attended exactly)."""
+    o = H.ocfg(B=1, Hkv=2, Hq=8, d=64, n_max=4096, T=16, L_blk=1024, update_interval=512, dtype="f32", iters=4)
+    K, V, _ = H.cache_for(o, 3000, comps=32, radius=None, sigma=0.3, seed=4)
+    oidx = mp.build_index(K, V, 2500, o)
+    assert not mp.cluster_update(oidx, K[:, :, 2500:2900], V[:, :, 2500:2900])
+    assert oidx["n_tokens"] == 2900 and oidx["n_clustered"] == 2500
+    Q = synth.make_queries(1, 1, 8, 64, "f32", seed=2)[0]
+    for budget in (1, 64, 2500):
+        run_decode(o, oidx, Q, budget)
+
+
+def test_singleton_clusters_equal_dense_attention():
+    o = H.ocfg(B=1, Hkv=1, Hq=4, d=128, n_max=512, T=1, L_blk=512, dtype="f32")
+    K, V, lab = H.cache_for(o, 512, comps=16, seed=1)
+    oidx = mp.index_from_assignment(K, V, 512, o, np.broadcast_to(np.arange(512), (1, 1, 512)))
+    Q = synth.make_queries(1, 1, 4, 128, "f32", seed=1)[0]
+    _, O, _ = run_decode(o, oidx, Q, 7)
+    dense = mp.dense_attention(Q, K, V, 512, 1)
+    assert np.abs(O - dense).max() <= 1e-4
+
+
+def test_large_logits_stay_finite():
+    o = H.ocfg(B=1, Hkv=2, Hq=8, d=128, n_max=2048, L_blk=2048)
+    K, V, lab = H.cache_for(o, 2048, comps=64, seed=6)
+    oidx = H.component_index(o, K, V, lab, 2048)
+    Q = synth.make_queries(1, 1, 8, 128, "bf16", seed=7, scale=1e3)[0]
+    for budget in (1, 200, 5000):
+        _, O, _ = run_decode(o, oidx, Q, budget)
+        assert np.isfinite(O).all()
+
+
+@pytest.mark.parametrize("coarse_budget", [64, 600, 100000])
+@pytest.mark.parametrize("budget", [1, 100, 100000])
+@pytest.mark.parametrize("no_approx", [False, True])
+def test_hierarchical_decode_matches_oracle(coarse_budget, budget, no_approx):
+    o = H.ocfg(B=2, Hkv=2, Hq=8, d=128, n_max=6000, T=16, L_blk=2048, levels=2, Tc=128)
+    K, V, lab = H.cache_for(o, 5500, comps=96, seed=9)
+    oidx = H.component_index(o, K, V, lab, 5500)
+    Q = synth.make_queries(1, 2, 8, 128, "bf16", seed=3)[0]
+    run_decode(o, oidx, Q, budget, coarse_budget=coarse_budget, no_approx=no_approx)

@@ -1,0 +1,420 @@
+#!/usr/bin/env python3
+"""Benchmark of the multipole-attention decode step on B200.
+
+Workload (default): batch 16, 8 KV / 32 query heads, head_dim 128, 32768 cached
+tokens per sequence, token budget 1638 (5% of the context, "95% sparsity"),
+seeded Gaussian-mixture keys (1 centroid per 16 tokens, 8K-token clustering
+blocks), bf16.  One step = one decode step of one attention layer for the
+whole batch (centroid pass, selection, token pass, combine).
+
+Reports algorithmic HBM GB/s (the bytes the method must read: all key and value
+centroids, the run offsets, the selected clusters' keys and values, the
+unclustered tail, Q and O) per device-timed step, with the L2 flushed between
+steps.  `--impl reference` times the CPU oracle instead (a bounded sample per
+step on the host cores).  N > 1: one process per GPU (torchrun), each decoding
+its own batch (weak scaling); time = max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attention µs/step & HBM GB/s (% roofline), B=16, 32K ctx, 95% sparsity"
+UNIT = "GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    """Measured roofline denominators, else the pool's earlier measurement."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def aggregate(local_value_sum, local_time, dist=None):
+    """(sum over ranks of the work, max over ranks of the time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return local_value_sum, local_time
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    w = torch.tensor([float(local_value_sum)], dtype=torch.float64, device=dev)
+    t = torch.tensor([float(local_time)], dtype=torch.float64, device=dev)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return w.item(), t.item()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def algorithmic_bytes_unit(w, C, n_sel_tokens, n_tail):
+    """Bytes one (batch, KV head) step must read or write (bf16 elements of 2 bytes):
+    all key and value centroids, the run offsets, the selected tokens' keys and
+    values, the tail's keys and values, the group's queries and outputs."""
+    e = 2 if w["dtype"] == "bf16" else 4
+    d, G = w["d"], w["Hq"] // w["Hkv"]
+    return 2 * C * d * e + (C + 1) * 4 + 2 * (n_sel_tokens + n_tail) * d * e + 2 * G * d * e
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+def oracle_units(w, k, seed):
+    """k (batch, KV head) units of the workload with oracle indices.
+
+    Clusters are the mixture components of each 8K block (a stand-in for the
+    k-means result: the decode cost does not depend on how clusters were found).
+    """
+    from clustered_sparse_decode_b200 import synth
+    from oracle import multipole as mp
+    rng = np.random.default_rng(seed)
+    n, d, G = w["n"], w["d"], w["Hq"] // w["Hkv"]
+    o = dict(B=1, Hkv=1, Hq=G, d=d, n_max=n, T=w["T"], L_blk=w["L_blk"], levels=1, Tc=w.get("Tc", 128),
+             iters=w["iters"], update_interval=w.get("update_interval", 1024), dtype=w["dtype"], seed=0)
+    units = []
+    for _ in range(k):
+        K, V, lab = synth.make_cache(1, 1, n, d, w["comps"], w["sigma"], radius=w["radius"],
+                                     outliers=w["outliers"], dtype=w["dtype"], seed=int(rng.integers(1 << 30)))
+        a = synth.component_assignment(lab, n, w["L_blk"], w["T"])
+        idx = mp.index_from_assignment(K, V, n, o, a)
+        units.append((idx, int(np.count_nonzero(np.diff(idx["off"][0, 0])))))
+    return units
+
+
+def time_oracle(w, units, seconds, seed):
+    """Time the oracle's decode over the units, fresh queries each, until `seconds` of decode time.
+
+    Returns (algorithmic bytes, decode seconds, unit-steps)."""
+    from clustered_sparse_decode_b200 import synth
+    from oracle import multipole as mp
+    try:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(1)
+    except ImportError:
+        ctx = None
+    rng = np.random.default_rng(seed)
+    d, G = w["d"], w["Hq"] // w["Hkv"]
+    tot_bytes, tot_time, pairs = 0, 0.0, 0
+    while tot_time < seconds:
+        idx, C = units[pairs % len(units)]
+        Q = synth.make_queries(1, 1, G, d, w["dtype"], seed=int(rng.integers(1 << 30)))[0]
+        info = {}
+        t0 = time.perf_counter()
+        mp.decode(idx, Q, w["budget"], info=info)
+        tot_time += time.perf_counter() - t0
+        nsel = int(np.sum(np.diff(idx["off"][0, 0])[info[(0, 0)]["sel"]]))
+        tot_bytes += algorithmic_bytes_unit(w, C, nsel, 0)
+        pairs += 1
+    if ctx is not None and hasattr(ctx, "restore_original_limits"):
+        ctx.restore_original_limits()
+    return tot_bytes, tot_time, pairs
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    units = w["B"] * w["Hkv"]
+    sample_units = oracle_units(w, 2, seed=1)
+    per_step = []
+    tot_b = tot_t = 0.0
+    pairs = 0
+    for s in range(args.warmup + args.steps):
+        b, t, p = time_oracle(w, sample_units, args.ref_seconds_per_step, seed=1000 + s)
+        if s >= args.warmup:
+            tot_b, tot_t, pairs = tot_b + b, tot_t + t, pairs + p
+            per_step.append(t / p * units)          # seconds for all units of one step
+    gbs = tot_b / tot_t / 1e9
+    ms = 1e3 * statistics.mean(per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, args),
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "value": gbs, "unit": UNIT,
+                         "sample": f"{pairs} (batch, KV head) decode steps of the workload, "
+                                   f"~{args.ref_seconds_per_step:.0f} s per step, extrapolated to "
+                                   f"{units} heads x batch per step"},
+        "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, args):
+    return {"workload": args.workload, "batch": w["B"], "kv_heads": w["Hkv"], "q_heads": w["Hq"],
+            "head_dim": w["d"], "context": w["n"], "budget": w["budget"], "tokens_per_centroid": w["T"],
+            "block_tokens": w["L_blk"], "levels": w.get("levels", 1), "kmeans_iters": w["iters"],
+            "l2": "flushed between timed steps (write of 2x L2)", "parallelism": f"dp{args.gpus} (independent batches)"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from clustered_sparse_decode_b200 import Config, MultipoleIndex, synth
+    from clustered_sparse_decode_b200 import build as libbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    libbuild.build()
+    dev = torch.device("cuda", local)
+    B, Hkv, Hq, d, n = w["B"], w["Hkv"], w["Hq"], w["d"], w["n"]
+    tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+
+    # inputs: seeded synthetic caches (distinct per rank), clustered on the GPU
+    K, V, _ = synth.make_cache(B, Hkv, n, d, w["comps"], w["sigma"], radius=w["radius"], outliers=w["outliers"],
+                               dtype=w["dtype"], seed=w["seed"] + 100 * rank)
+    Kd = torch.from_numpy(K).to(dev).to(tdt)
+    Vd = torch.from_numpy(V).to(dev).to(tdt)
+    del K, V
+    cfg = Config(batch=B, kv_heads=Hkv, q_heads=Hq, head_dim=d, max_tokens=n, tokens_per_centroid=w["T"],
+                 block_tokens=w["L_blk"], levels=w.get("levels", 1), coarse_tokens_per_centroid=w.get("Tc", 128),
+                 kmeans_iters=w["iters"], dtype=w["dtype"], seed=w["seed"])
+    idx = MultipoleIndex(cfg, device=dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    idx.build(Kd, Vd)
+    torch.cuda.synchronize()
+    build_s = time.perf_counter() - t0
+    del Kd, Vd
+    if idx.check_device_error() != 0:
+        raise RuntimeError("device error after build")
+    nq = args.warmup + args.steps
+    Qh = synth.make_queries(nq, B, Hq, d, w["dtype"], seed=w["seed"] + 7 + 100 * rank)
+    Q = torch.from_numpy(Qh).to(dev).to(tdt)
+    O = torch.empty((B, Hq, d), dtype=tdt, device=dev)
+    budget = w["budget"]
+    cb = w.get("coarse_budget", 0)
+
+    # algorithmic bytes of each timed step, from its actual selection (untimed pass)
+    off = idx.arrays()["off"]
+    cnt = (off[:, :, 1:] - off[:, :, :-1]).to(torch.int64)
+    C_unit = (cnt > 0).sum(dim=2)                                     # [B, Hkv]
+    mask = torch.zeros((B, Hkv, idx.slots), dtype=torch.uint8, device=dev)
+    step_bytes = []
+    for s in range(args.warmup, nq):
+        idx.decode(Q[s], budget, coarse_budget=cb, out=O, sel_mask=mask)
+        nsel = (cnt * mask.to(torch.int64)).sum(dim=2)                # [B, Hkv]
+        tot = 0
+        for b in range(B):
+            for h in range(Hkv):
+                tot += algorithmic_bytes_unit(w, int(C_unit[b, h]), int(nsel[b, h]), 0)
+        step_bytes.append(tot)
+    sel_tokens_mean = float(nsel.float().mean())
+
+    # L2 flush buffer and per-step / per-phase events
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    n_ph = 5 if cfg.levels == 1 else 7
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ph)] for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    for s in range(args.warmup):
+        flush.zero_()
+        idx.decode(Q[s], budget, coarse_budget=cb, out=O)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        idx.decode(Q[args.warmup + i], budget, coarse_budget=cb, out=O, phase_events=ev[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
+    phase_ms = [statistics.mean(ev[i][p].elapsed_time(ev[i][p + 1]) for i in range(args.steps))
+                for p in range(n_ph - 1)]
+    local_time = sum(step_ms) / 1e3
+    local_bytes = sum(step_bytes)
+    tot_bytes, tot_time = aggregate(local_bytes, local_time, dist)
+    gbs = tot_bytes / tot_time / 1e9
+    ms_per_step = 1e3 * tot_time / args.steps
+
+    # end to end through the C ABI: Q from pinned host memory, O back to the host, every step
+    Qpin = torch.from_numpy(Qh).to(tdt).pin_memory() if w["dtype"] == "bf16" else torch.from_numpy(Qh).pin_memory()
+    Opin = torch.empty((B, Hq, d), dtype=tdt).pin_memory()
+    Qdev = torch.empty((B, Hq, d), dtype=tdt, device=dev)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Qdev.copy_(Qpin[i], non_blocking=True)
+        idx.decode(Qdev, budget, coarse_budget=cb, out=O)
+        Opin.copy_(O, non_blocking=True)
+        b_.record(stream)
+        b_.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b_))
+    e2e_bytes, e2e_time = aggregate(local_bytes, sum(e2e_ms) / 1e3, dist)
+    qbytes = B * Hq * d * (2 if w["dtype"] == "bf16" else 4)
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    names = ["centroid pass", "select", "token pass", "combine"] if cfg.levels == 1 else \
+        ["coarse pass", "coarse select", "fine pass", "fine select", "token pass", "combine"]
+    dom = int(np.argmax(phase_ms))
+    e = 2 if w["dtype"] == "bf16" else 4
+    C_tot = int(C_unit.sum())
+    sel_tot = sum(step_bytes) / len(step_bytes)
+    phase_alg = {
+        "centroid pass": 2 * C_tot * d * e + (idx.slots + 1) * 4 * B * Hkv,
+        "token pass": sel_tot - (2 * C_tot * d * e + (idx.slots + 1) * 4 * B * Hkv) - 2 * B * Hq * d * e,
+    }
+    dom_name = names[dom]
+    dom_bytes = phase_alg.get(dom_name)
+    roof = None
+    if dom_bytes is not None:
+        ach = dom_bytes / (phase_ms[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(dom_name, args.workload),
+                "kernel": dom_name, "peak_source": pk["source"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b_, t_, p_ = time_oracle(w, oracle_units(w, 2, seed=1), args.cpu_seconds, seed=99)
+        cpu = {"value": b_ / t_ / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{p_} (batch, KV head) decode steps of the workload on one host core (~{args.cpu_seconds:.0f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+            "config": config_dict(w, args),
+            "us_per_step": 1e3 * ms_per_step, "tokens_per_s": w["B"] * world * args.steps / tot_time,
+            "pct_hbm_roofline": gbs / world / pk["hbm_gbs"],
+            "roofline": roof,
+            "phases_ms": dict(zip(names, phase_ms)),
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_bytes / e2e_time / 1e9, "unit": UNIT, "h2d_bytes_per_step": qbytes,
+                    "d2h_bytes_per_step": qbytes},
+            "gpu_launches": args.steps * (4 if cfg.levels == 1 else 7),
+            "clocks": clk,
+            "build_s": build_s,
+            "selected_tokens_per_head": sel_tokens_mean,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if current."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        parts = [x.strip() for x in line.strip().strip("|").split("|")]
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload:
+            try:
+                if parts[3] != source_digest():
+                    return None
+                return float(parts[2])
+            except ValueError:
+                return None
+    return None
+
+
+def source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "clustered_sparse_decode_b200", "csrc"))):
+        h.update(open(os.path.join(ROOT, "clustered_sparse_decode_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="batch16_32k_sparse95")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds-per-step", type=float, default=1.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from clustered_sparse_decode_b200 import synth
+    w = synth.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -40,7 +40,9 @@ class MpDecodeParams(ctypes.Structure):
     _fields_ = [("budget", ctypes.c_int32), ("coarse_budget", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("flags", ctypes.c_uint32), ("n_split", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("sel_mask_out", ctypes.c_void_p), ("coarse_sel_mask_out", ctypes.c_void_p),
-                ("scores_out", ctypes.c_void_p), ("coarse_scores_out", ctypes.c_void_p)]
+                ("scores_out", ctypes.c_void_p), ("coarse_scores_out", ctypes.c_void_p),
+                ("phase_events", ctypes.c_void_p), ("n_phase_events", ctypes.c_int32),
+                ("reserved2", ctypes.c_int32)]
 
 
 _lib = None

@@ -134,11 +134,13 @@ class MultipoleIndex:
         return bool(fired.value)
 
     def decode(self, Q, budget, coarse_budget=0, scale=0.0, no_approx=False, n_split=0, out=None,
-               sel_mask=None, coarse_sel_mask=None, scores=None, coarse_scores=None, stream=None):
+               sel_mask=None, coarse_sel_mask=None, scores=None, coarse_scores=None, phase_events=None,
+               stream=None):
         """One decode step: O [B, Hq, d] for Q [B, Hq, d] (mp_decode).
 
         Optional device outputs: sel_mask / coarse_sel_mask (uint8 [B, Hkv, slots]),
-        scores / coarse_scores (float32 [B, Hkv, slots]).
+        scores / coarse_scores (float32 [B, Hkv, slots]).  phase_events: torch.cuda.Event
+        objects (already recorded once) that the library records at its kernel boundaries.
         """
         c = self.cfg
         want = (c.batch, c.q_heads, c.head_dim)
@@ -157,6 +159,12 @@ class MultipoleIndex:
         p.coarse_sel_mask_out = coarse_sel_mask.data_ptr() if coarse_sel_mask is not None else None
         p.scores_out = scores.data_ptr() if scores is not None else None
         p.coarse_scores_out = coarse_scores.data_ptr() if coarse_scores is not None else None
+        evs = None
+        if phase_events:
+            evs = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
+            p.phase_events = ctypes.cast(evs, ctypes.c_void_p)
+            p.n_phase_events = len(phase_events)
+        p.reserved2 = 0
         L.check(self.lib.mp_decode(ctypes.byref(self.h), _ptr(Q), _ptr(out), ctypes.byref(p), _ptr(self.scratch),
                                    self.scratch.numel(), _stream(stream)), "mp_decode")
         return out

@@ -175,7 +175,8 @@ mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode
   mp_status s = check_index(idx);
   if (s != MP_OK) return s;
   if (!Q || !O || !p || !d_scratch) return MP_EINVAL;
-  if (p->reserved != 0 || p->n_split < 0 || p->n_split > 64) return MP_EINVAL;
+  if (p->reserved != 0 || p->reserved2 != 0 || p->n_split < 0 || p->n_split > 64) return MP_EINVAL;
+  if (p->n_phase_events < 0 || (p->n_phase_events > 0 && !p->phase_events)) return MP_EINVAL;
   if (!std::isfinite(p->scale)) return MP_EINVAL;
   if ((p->flags & ~MP_NO_APPROX) != 0) return MP_EINVAL;
   return decode_impl(idx, Q, O, p, d_scratch, scratch_bytes, static_cast<cudaStream_t>(stream));

@@ -152,6 +152,7 @@ pass_kernel(PassArgs a) {
       if (nruns < 0 || nruns > L.rl.cap || total < 0) { set_error(a.err, E_BAD_LIST); total = 0; }
       if (nruns <= 0) total = 0;
     }
+    if (L.shat && total > L.shat_cap) { set_error(a.err, E_BAD_LIST); total = L.shat_cap; }
     const int per = (total + nsplit - 1) / nsplit;
     const int r0 = min(total, split * per), r1 = min(total, r0 + per);
     const T* Kb = reinterpret_cast<const T*>(L.K) + (size_t)unit * L.unit_rows * D;
@@ -341,7 +342,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
       int y = __shfl_up_sync(kFull, w, o);
       if (lane >= o) w += y;
     }
-    s_warp[lane] = w;   // inclusive over warps
+    if (lane < NT / kWarp) s_warp[lane] = w;   // inclusive over warps
   }
   __syncthreads();
   int before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
@@ -671,6 +672,11 @@ static cudaError_t launch_combine(int dtype, int D, const float* pm, const float
   return cudaGetLastError();
 }
 
+static void record_phase(const mp_decode_params* prm, int i, cudaStream_t st) {
+  if (i < prm->n_phase_events && prm->phase_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(prm->phase_events[i]), st);
+}
+
 mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
                       void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const mp_config& c = idx->cfg;
@@ -730,6 +736,8 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
   SelectArgs sa{};
   sa.off = off; sa.coff = coff; sa.slots = idx->slots; sa.coarse_slots = idx->coarse_slots; sa.err = err;
 
+  int ev = 0;
+  record_phase(prm, ev++, st);
   if (c.levels == 1) {
     // 1. all centroids
     PassArgs p1 = pa_args;
@@ -739,6 +747,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
     ce = launch_pass_any(c.dtype, D, G, p1, L.nsplit_c, units, st);
     part_used += L.nsplit_c;
     if (ce != cudaSuccess) return MP_ECUDA;
+    record_phase(prm, ev++, st);
     // 2. select
     sa.implicit_n = idx->slots;
     sa.shat = shat; sa.shat_cap = idx->slots;
@@ -751,6 +760,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
     sa.scores_out = prm->scores_out;
     ce = launch_select(sa, units, st);
     if (ce != cudaSuccess) return MP_ECUDA;
+    record_phase(prm, ev++, st);
   } else {
     RunList fine = runlist_at(base, L.o_fine, L.cap_fine);
     RunList csub = runlist_at(base, L.o_csub, L.cap_csub);
@@ -765,6 +775,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
     ce = launch_pass_any(c.dtype, D, G, p1, L.nsplit_c, units, st);
     part_used += L.nsplit_c;
     if (ce != cudaSuccess) return MP_ECUDA;
+    record_phase(prm, ev++, st);
     // 2. coarse select -> fine candidate ranges
     SelectArgs s1 = sa;
     s1.implicit_n = idx->coarse_slots;
@@ -778,6 +789,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
     s1.scores_out = prm->coarse_scores_out;
     ce = launch_select(s1, units, st);
     if (ce != cudaSuccess) return MP_ECUDA;
+    record_phase(prm, ev++, st);
     // 3. fine centroids under selected coarse clusters, minus the selected coarse terms
     PassArgs p2 = pa_args;
     p2.n_lists = approx ? 2 : 1;
@@ -787,6 +799,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
     ce = launch_pass_any(c.dtype, D, G, p2, L.nsplit_f, units, st);
     part_used += L.nsplit_f;
     if (ce != cudaSuccess) return MP_ECUDA;
+    record_phase(prm, ev++, st);
     // 4. fine select -> token runs
     SelectArgs s2 = sa;
     s2.implicit_n = 0;
@@ -801,6 +814,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
     s2.scores_out = prm->scores_out;
     ce = launch_select(s2, units, st);
     if (ce != cudaSuccess) return MP_ECUDA;
+    record_phase(prm, ev++, st);
   }
   // 5. exact tokens, minus the selected centroid terms
   PassArgs p3 = pa_args;
@@ -811,8 +825,10 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
   ce = launch_pass_any(c.dtype, D, G, p3, nsplit_t, units, st);
   part_used += nsplit_t;
   if (ce != cudaSuccess) return MP_ECUDA;
+  record_phase(prm, ev++, st);
   // 6. combine the partials written by this call
   ce = launch_combine(c.dtype, D, pm, pl, pa, L.P, part_used, O, units * G, st);
+  record_phase(prm, ev++, st);
   (void)es;
   return ce == cudaSuccess ? MP_OK : MP_ECUDA;
 }

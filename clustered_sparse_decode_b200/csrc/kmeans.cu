@@ -103,7 +103,7 @@ __device__ double block_scan_f64(double v, double* s_w, double* total) {
       double y = __shfl_up_sync(kFull, w, o);
       if (lane >= o) w += y;
     }
-    s_w[lane] = w;
+    if (lane < NT / kWarp) s_w[lane] = w;
   }
   __syncthreads();
   double before = (warp > 0 ? s_w[warp - 1] : 0.0) + (x - v);
@@ -130,7 +130,7 @@ __device__ int block_scan_i32(int v, int* s_w, int* total) {
       int y = __shfl_up_sync(kFull, w, o);
       if (lane >= o) w += y;
     }
-    s_w[lane] = w;
+    if (lane < NT / kWarp) s_w[lane] = w;
   }
   __syncthreads();
   int before = (warp > 0 ? s_w[warp - 1] : 0) + x - v;

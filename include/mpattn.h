@@ -131,6 +131,14 @@ typedef struct {
   float* scores_out;        /* optional [B, H, slots]: group score max_g scale*q_g.Kc of every
                                scored non-empty fine cluster, -inf elsewhere */
   float* coarse_scores_out; /* optional [B, H, coarse_slots] (levels == 2) */
+  void** phase_events;      /* optional: n_phase_events cudaEvent_t handles (created by the caller)
+                               recorded on `stream` at the kernel boundaries of the step, in order:
+                               flat:   start | centroid pass | select | token pass | combine
+                               levels 2: start | coarse pass | coarse select | fine pass |
+                                         fine select | token pass | combine
+                               (5 resp. 7 events; extra handles are not touched) */
+  int32_t n_phase_events;
+  int32_t reserved2;        /* must be 0 */
 } mp_decode_params;
 
 /* Workspace sizes for `cfg`.  index_bytes: the index and the scratch its

@@ -42,7 +42,7 @@ def test_struct_layout_matches_the_header(tmp_path):
                      "workspace_bytes", "layout"],
         "mp_index_view": ["Kc", "coff"],
         "mp_decode_params": ["budget", "scale", "flags", "n_split", "reserved", "sel_mask_out",
-                             "coarse_scores_out"],
+                             "coarse_scores_out", "phase_events", "n_phase_events", "reserved2"],
     }
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "mpattn.h"', "int main(void){"]
     for s, fs in fields.items():

@@ -122,6 +122,9 @@ WORKLOADS = {
     "batch16_32k_sparse95": dict(B=16, Hkv=8, Hq=32, d=128, n=32768, comps=512, sigma=0.25,
                                  radius=(1.0, 4.0), outliers=(4, 4.0), dtype="bf16", T=16,
                                  L_blk=8192, budget=1638, iters=10, steps=64, seed=3000),
+    "batch4_32k_sparse95": dict(B=4, Hkv=8, Hq=32, d=128, n=32768, comps=512, sigma=0.25,
+                                radius=(1.0, 4.0), outliers=(4, 4.0), dtype="bf16", T=16,
+                                L_blk=8192, budget=1638, iters=10, steps=64, seed=3500),
     "hier_64k": dict(B=4, Hkv=8, Hq=32, d=128, n=65536, comps=512, sigma=0.25, radius=(1.0, 4.0),
                      outliers=(4, 4.0), dtype="bf16", T=16, L_blk=8192, budget=512, levels=2, Tc=128,
                      coarse_budget=4096, iters=10, steps=64, seed=4000),

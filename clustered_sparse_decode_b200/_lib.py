@@ -9,8 +9,10 @@ MP_OK, MP_EINVAL, MP_ENOSPC, MP_ECUDA, MP_EUNSUPPORTED, MP_EDEVICE = range(6)
 MP_F32, MP_BF16 = 0, 1
 MP_INIT_KMEANSPP, MP_INIT_STRIDE = 0, 1
 MP_NO_APPROX = 1
+MP_STATIC_SCRATCH_BYTES = 32 << 20
 
 EXPORTS = ["mp_workspace_size", "mp_index_init", "mp_cluster_build", "mp_cluster_update", "mp_decode",
+           "mp_decode_static",
            "mp_index_export", "mp_index_import", "mp_check_device_error", "mp_status_str"]
 
 
@@ -71,6 +73,7 @@ def load():
         "mp_cluster_build": [P(MpIndex), vp, vp, i32, vp, vp],
         "mp_cluster_update": [P(MpIndex), vp, vp, i32, P(i32), vp],
         "mp_decode": [P(MpIndex), vp, vp, P(MpDecodeParams), vp, sz, vp],
+        "mp_decode_static": [P(MpIndex), vp, vp, P(MpDecodeParams), vp],
         "mp_index_export": [P(MpIndex), P(MpIndexView)],
         "mp_index_import": [P(MpIndex), P(MpIndexView), i64, i64, vp],
         "mp_check_device_error": [P(MpIndex), P(i32), vp],

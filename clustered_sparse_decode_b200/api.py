@@ -169,6 +169,31 @@ class MultipoleIndex:
                                    self.scratch.numel(), _stream(stream)), "mp_decode")
         return out
 
+    def decode_static(self, Q, budget, coarse_budget=0, scale=0.0, no_approx=False, n_split=0, out=None,
+                      stream=None):
+        """decode() without the index's scratch tensor (mp_decode_static).
+
+        For callers that cannot allocate device memory when they decode: the
+        library's own fixed 32 MiB device array serves as scratch.  Calls that
+        overlap on the GPU race on that array; the first call on a device should
+        come before any stream capture.
+        """
+        c = self.cfg
+        want = (c.batch, c.q_heads, c.head_dim)
+        if tuple(Q.shape) != want or Q.dtype != c.torch_dtype or not Q.is_contiguous():
+            raise ValueError(f"Q must be a contiguous {c.torch_dtype} tensor of shape {want}")
+        if out is None:
+            out = torch.empty_like(Q)
+        p = L.MpDecodeParams()
+        p.budget = int(budget)
+        p.coarse_budget = int(coarse_budget)
+        p.scale = float(scale)
+        p.flags = L.MP_NO_APPROX if no_approx else 0
+        p.n_split = int(n_split)
+        L.check(self.lib.mp_decode_static(ctypes.byref(self.h), _ptr(Q), _ptr(out), ctypes.byref(p),
+                                          _stream(stream)), "mp_decode_static")
+        return out
+
     def arrays(self):
         """Views (torch tensors) of the index arrays inside the workspace (mp_index_export)."""
         v = L.MpIndexView()

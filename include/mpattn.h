@@ -194,6 +194,29 @@ mp_status mp_cluster_update(mp_index* idx, const void* K_new, const void* V_new,
 mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
                     void* d_scratch, size_t scratch_bytes, void* stream);
 
+/* Size of the library's own decode scratch used by mp_decode_static. */
+#define MP_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* mp_decode for callers that cannot allocate device memory (no counterpart in
+ * the paper: an interface addition).  A serving engine that gives all free
+ * device memory to its own KV-cache pool at start-up has none left for the
+ * decode scratch, and on a latency-critical path cudaMalloc / cudaFree may
+ * synchronise the device.  Same arguments, semantics and results as
+ * mp_decode, except that the scratch is a fixed array of
+ * MP_STATIC_SCRATCH_BYTES (32 MiB) inside the library, which every device that
+ * loads the library holds until the process exits.  It calls no allocator.
+ *  - Returns MP_ENOSPC if the configuration's decode_scratch_bytes
+ *    (mp_workspace_size) exceed MP_STATIC_SCRATCH_BYTES.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls that overlap on
+ *    the GPU (other streams, other threads, other indices) race on it: order
+ *    them, e.g. on one stream. */
+mp_status mp_decode_static(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
+                           void* stream);
+
 /* Device pointers of the index arrays (layouts above). */
 mp_status mp_index_export(const mp_index* idx, mp_index_view* view);
 

@@ -267,7 +267,8 @@ def run_ours(args, w):
     # L2 flush buffer and per-step / per-phase events
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-    n_ph = 5 if cfg.levels == 1 else 7
+    names = idx.decode_phases()
+    n_ph = len(names) + 1
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ph)] for _ in range(args.steps)]
     for row in ev:
@@ -321,13 +322,12 @@ def run_ours(args, w):
 
     # roofline of the dominant kernel
     pk = peaks()
-    names = ["centroid pass", "select", "token pass", "combine"] if cfg.levels == 1 else \
-        ["coarse pass", "coarse select", "fine pass", "fine select", "token pass", "combine"]
     dom = int(np.argmax(phase_ms))
     e = 2 if w["dtype"] == "bf16" else 4
     C_tot = int(C_unit.sum())
     sel_tot = sum(step_bytes) / len(step_bytes)
     phase_alg = {
+        "centroid pass + value pass": sel_tot,
         "centroid pass": 2 * C_tot * d * e + (idx.slots + 1) * 4 * B * Hkv,
         "token pass": sel_tot - (2 * C_tot * d * e + (idx.slots + 1) * 4 * B * Hkv) - 2 * B * Hq * d * e,
     }
@@ -359,7 +359,7 @@ def run_ours(args, w):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_bytes / e2e_time / 1e9, "unit": UNIT, "h2d_bytes_per_step": qbytes,
                     "d2h_bytes_per_step": qbytes},
-            "gpu_launches": args.steps * (4 if cfg.levels == 1 else 7),
+            "gpu_launches": args.steps * (2 if names[-1] == "centroid pass + value pass" else len(names)),
             "clocks": clk,
             "build_s": build_s,
             "selected_tokens_per_head": sel_tokens_mean,

@@ -102,6 +102,20 @@ class MultipoleIndex:
     def coarse_slots(self):
         return self.h.coarse_slots
 
+    def decode_phases(self):
+        """Names of the intervals between the phase events that decode() records for this index.
+
+        A flat bf16 index with at most 4096 slots per unit decodes with a
+        centroid pass and a value pass (after a reset of its ticket words); the
+        others run a longer kernel pipeline.
+        """
+        c = self.cfg
+        if c.levels == 1 and c.dtype == "bf16" and self.slots <= 4096:
+            return ["ticket reset", "centroid pass + value pass"]
+        if c.levels == 1:
+            return ["centroid pass", "select", "token pass", "combine"]
+        return ["coarse pass", "coarse select", "fine pass", "fine select", "token pass", "combine"]
+
     def _check_kv(self, t, n):
         c = self.cfg
         want = (c.batch, c.kv_heads, n, c.head_dim)

@@ -608,8 +608,14 @@ static DecodeLayout decode_layout(const mp_config& c, int slots, int coarse_slot
   return L;
 }
 
+size_t stream_scratch_bytes(const mp_config& c, int slots);
+bool stream_supported(const mp_config& c, int slots);
+mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
+                        size_t scratch_bytes, float scale, cudaStream_t st);
+
+// Both decode paths place their scratch from the start of the buffer; one call uses one of them.
 size_t decode_scratch_bytes(const mp_config& c, int slots, int coarse_slots) {
-  return decode_layout(c, slots, coarse_slots).bytes;
+  return std::max(decode_layout(c, slots, coarse_slots).bytes, stream_scratch_bytes(c, slots));
 }
 
 static RunList runlist_at(char* base, const size_t o[3], int cap) {
@@ -680,6 +686,11 @@ static void record_phase(const mp_decode_params* prm, int i, cudaStream_t st) {
 mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
                       void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const mp_config& c = idx->cfg;
+  // flat bf16 index: the one-kernel streaming path (decode_stream.cu)
+  if (stream_supported(c, idx->slots)) {
+    const float sc = prm->scale != 0.f ? prm->scale : 1.0f / sqrtf((float)c.head_dim);
+    return stream_decode(idx, Q, O, prm, scratch, scratch_bytes, sc, st);
+  }
   DecodeLayout L = decode_layout(c, idx->slots, idx->coarse_slots);
   if (scratch_bytes < L.bytes) return MP_ENOSPC;
   char* base = static_cast<char*>(scratch);

@@ -133,10 +133,11 @@ typedef struct {
   float* coarse_scores_out; /* optional [B, H, coarse_slots] (levels == 2) */
   void** phase_events;      /* optional: n_phase_events cudaEvent_t handles (created by the caller)
                                recorded on `stream` at the kernel boundaries of the step, in order:
-                               flat:   start | centroid pass | select | token pass | combine
-                               levels 2: start | coarse pass | coarse select | fine pass |
-                                         fine select | token pass | combine
-                               (5 resp. 7 events; extra handles are not touched) */
+                               flat bf16, slots <= 4096: start | ticket reset | centroid pass + value pass
+                               other flat:  start | centroid pass | select | token pass | combine
+                               levels 2:    start | coarse pass | coarse select | fine pass |
+                                            fine select | token pass | combine
+                               (3, 5 resp. 7 events; extra handles are not touched) */
   int32_t n_phase_events;
   int32_t reserved2;        /* must be 0 */
 } mp_decode_params;

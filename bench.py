@@ -238,9 +238,10 @@ def run_ours(args, w):
     idx.build(Kd, Vd)
     torch.cuda.synchronize()
     build_s = time.perf_counter() - t0
-    del Kd, Vd
     if idx.check_device_error() != 0:
         raise RuntimeError("device error after build")
+    kassign = time_assign(idx, Kd, w, args) if not args.no_assign else None
+    del Kd, Vd
     nq = args.warmup + args.steps
     Qh = synth.make_queries(nq, B, Hq, d, w["dtype"], seed=w["seed"] + 7 + 100 * rank)
     Q = torch.from_numpy(Qh).to(dev).to(tdt)
@@ -362,6 +363,7 @@ def run_ours(args, w):
             "gpu_launches": args.steps * (2 if names[-1] == "centroid pass + value pass" else len(names)),
             "clocks": clk,
             "build_s": build_s,
+            "kmeans_assign": kassign,
             "selected_tokens_per_head": sel_tokens_mean,
         }
         print(json.dumps(line), flush=True)
@@ -369,6 +371,45 @@ def run_ours(args, w):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def assign_flops(w):
+    """Algorithmic flops of one assignment step: 2 L_j C_j d per (unit, block), C_j = ceil(L_j / T)."""
+    n, Lb, T, d = w["n"], w["L_blk"], w["T"], w["d"]
+    f = 0
+    for j in range(-(-n // Lb)):
+        L = min(n, (j + 1) * Lb) - j * Lb
+        f += 2 * L * (-(-L // T)) * d
+    return f * w["B"] * w["Hkv"]
+
+
+def time_assign(idx, Kd, w, args, reps=5, warm=3):
+    """One k-means assignment step over the whole index (one launch), CUDA events on the launching stream.
+
+    The keys (B x Hkv x n x d) are far larger than L2, so each step streams them from HBM.
+    """
+    import torch
+    out = torch.empty((w["B"], w["Hkv"], idx.n_clustered), dtype=torch.int32, device=Kd.device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warm):
+        idx.assign(Kd, out=out)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record(stream)
+    for i in range(reps):
+        idx.assign(Kd, out=out)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
+    if idx.check_device_error() != 0:
+        raise RuntimeError("device error after assignment")
+    flops = assign_flops(w)
+    pk = peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    return {"ms": ms, "flops_per_launch": flops, "tflops": tf, "bound": "tensor",
+            "peak": pk["bf16_tflops"], "frac": tf / pk["bf16_tflops"],
+            "frac_sustained": tf / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+            "peak_source": pk["source"], "dtype": w["dtype"]}
 
 
 def traffic_for(kernel, workload):
@@ -406,6 +447,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds-per-step", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-assign", action="store_true", help="skip the timed k-means assignment step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

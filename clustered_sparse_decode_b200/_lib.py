@@ -11,7 +11,8 @@ MP_INIT_KMEANSPP, MP_INIT_STRIDE = 0, 1
 MP_NO_APPROX = 1
 MP_STATIC_SCRATCH_BYTES = 32 << 20
 
-EXPORTS = ["mp_workspace_size", "mp_index_init", "mp_cluster_build", "mp_cluster_update", "mp_decode",
+EXPORTS = ["mp_workspace_size", "mp_index_init", "mp_cluster_build", "mp_cluster_update", "mp_cluster_assign",
+           "mp_decode",
            "mp_decode_static",
            "mp_index_export", "mp_index_import", "mp_check_device_error", "mp_status_str"]
 
@@ -72,6 +73,7 @@ def load():
         "mp_index_init": [P(MpConfig), vp, sz, P(MpIndex), vp],
         "mp_cluster_build": [P(MpIndex), vp, vp, i32, vp, vp],
         "mp_cluster_update": [P(MpIndex), vp, vp, i32, P(i32), vp],
+        "mp_cluster_assign": [P(MpIndex), vp, i32, vp, vp],
         "mp_decode": [P(MpIndex), vp, vp, P(MpDecodeParams), vp, sz, vp],
         "mp_decode_static": [P(MpIndex), vp, vp, P(MpDecodeParams), vp],
         "mp_index_export": [P(MpIndex), P(MpIndexView)],

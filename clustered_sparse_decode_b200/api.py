@@ -147,6 +147,24 @@ class MultipoleIndex:
                                            ctypes.byref(fired), _stream(stream)), "mp_cluster_update")
         return bool(fired.value)
 
+    def assign(self, K, out=None, stream=None):
+        """Nearest-centroid slot of every clustered key under the current centroids (mp_cluster_assign).
+
+        K: the index's keys [B, Hkv, n_clustered, d] in token order; returns
+        int32 [B, Hkv, n_clustered] global slots.
+        """
+        n = self.n_clustered
+        self._check_kv(K, n)
+        c = self.cfg
+        want = (c.batch, c.kv_heads, n)
+        if out is None:
+            out = torch.empty(want, dtype=torch.int32, device=self.device)
+        elif tuple(out.shape) != want or out.dtype != torch.int32 or not out.is_contiguous() or out.device != self.device:
+            raise ValueError(f"out must be a contiguous int32 tensor of shape {want} on {self.device}")
+        L.check(self.lib.mp_cluster_assign(ctypes.byref(self.h), _ptr(K), int(n), _ptr(out), _stream(stream)),
+                "mp_cluster_assign")
+        return out
+
     def decode(self, Q, budget, coarse_budget=0, scale=0.0, no_approx=False, n_split=0, out=None,
                sel_mask=None, coarse_sel_mask=None, scores=None, coarse_scores=None, phase_events=None,
                stream=None):

@@ -9,6 +9,7 @@ namespace mp {
 mp_status build_impl(mp_index* idx, const void* K, const void* V, int32_t n, const void* init, cudaStream_t st);
 mp_status update_impl(mp_index* idx, const void* K_new, const void* V_new, int32_t n_new, int32_t* fired,
                       cudaStream_t st);
+mp_status assign_impl(const mp_index* idx, const void* K, int32_t n, int32_t* out, cudaStream_t st);
 mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
                       size_t scratch_bytes, cudaStream_t st);
 size_t decode_scratch_bytes(const mp_config& c, int slots, int coarse_slots);
@@ -168,6 +169,13 @@ mp_status mp_cluster_update(mp_index* idx, const void* K_new, const void* V_new,
   if (n_new > 0 && (!K_new || !V_new)) return MP_EINVAL;
   if (idx->n_tokens + n_new > idx->cfg.max_tokens) return MP_ENOSPC;
   return update_impl(idx, K_new, V_new, n_new, reclustered, static_cast<cudaStream_t>(stream));
+}
+
+mp_status mp_cluster_assign(const mp_index* idx, const void* K, int32_t n, int32_t* assign_out, void* stream) {
+  mp_status s = check_index(idx);
+  if (s != MP_OK) return s;
+  if (n != idx->n_clustered || (n > 0 && (!K || !assign_out))) return MP_EINVAL;
+  return assign_impl(idx, K, n, assign_out, static_cast<cudaStream_t>(stream));
 }
 
 mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* p, void* d_scratch,

@@ -776,6 +776,13 @@ static BlockJob make_job(const mp_index* idx) {
   return b;
 }
 
+// The tensor-core assignment (assign_tc.cu) for bf16 keys.
+bool assign_tc_supported(int dtype, int D, int C_blk, const void* srcK, const void* Kc, int64_t src_rows_total,
+                         int64_t centroid_rows);
+cudaError_t launch_assign_tc(int D, const void* srcK, int64_t src_rows_total, int64_t src_unit_rows, int64_t src_row0,
+                             const void* Kc, int units, int slots, int blk0, int nbj, int L_blk, int T, int C_blk,
+                             int64_t n_total, int32_t* assign, int64_t max_tokens, int32_t* err, cudaStream_t st);
+
 template <typename T, int D>
 static cudaError_t run_lloyd(const BlockJob& b, int nbj, int units, int init_mode, int L_old_tokens,
                              const void* init, int levels, cudaStream_t st) {
@@ -802,8 +809,16 @@ static cudaError_t run_lloyd(const BlockJob& b, int nbj, int units, int init_mod
   if (e != cudaSuccess) return e;
   const int tiles = (b.L_blk + kAT - 1) / kAT;
   const int mean_blocks = (b.C_blk + 7) / 8;
+  const int64_t src_rows = (int64_t)units * b.src_unit_rows + b.src_row0;
+  const bool tc = assign_tc_supported(DT<T>::id, D, b.C_blk, b.srcK, b.Kc, src_rows, (int64_t)units * b.slots);
   for (int it = 0; it < b.iters; ++it) {
-    assign_simt_kernel<T, D><<<dim3(tiles, nbj, units), 256, smem_a, st>>>(b);
+    if (tc) {
+      e = launch_assign_tc(D, b.srcK, src_rows, b.src_unit_rows, b.src_row0, b.Kc, units, b.slots, b.blk0, nbj,
+                           b.L_blk, b.T, b.C_blk, b.n_total, b.assign, b.max_tokens, b.err, st);
+      if (e != cudaSuccess) return e;
+    } else {
+      assign_simt_kernel<T, D><<<dim3(tiles, nbj, units), 256, smem_a, st>>>(b);
+    }
     sort_kernel<<<gb, kSortThreads, smem_s, st>>>(b);
     mean_kernel<T, D, false><<<dim3(mean_blocks, nbj, units), 256, 0, st>>>(b);
   }
@@ -892,6 +907,47 @@ mp_status build_impl(mp_index* idx, const void* K, const void* V, int32_t n, con
   idx->n_tokens = n;
   idx->n_clustered = n;
   return MP_OK;
+}
+
+// One assignment step of every block of the index against its current
+// centroids: the job of a build over the caller's keys, with the output rows
+// [unit][n] of the caller's array.
+template <typename T, int D>
+static cudaError_t run_assign(const BlockJob& b, int nbj, int units, cudaStream_t st) {
+  const int64_t src_rows = (int64_t)units * b.src_unit_rows + b.src_row0;
+  if (assign_tc_supported(DT<T>::id, D, b.C_blk, b.srcK, b.Kc, src_rows, (int64_t)units * b.slots))
+    return launch_assign_tc(D, b.srcK, src_rows, b.src_unit_rows, b.src_row0, b.Kc, units, b.slots, b.blk0, nbj,
+                            b.L_blk, b.T, b.C_blk, b.n_total, b.assign, b.max_tokens, b.err, st);
+  const size_t smem_a = (size_t)(2 * D * kALD + kAT) * sizeof(float);
+  cudaError_t e =
+      cudaFuncSetAttribute(assign_simt_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+  if (e != cudaSuccess) return e;
+  assign_simt_kernel<T, D><<<dim3((b.L_blk + kAT - 1) / kAT, nbj, units), 256, smem_a, st>>>(b);
+  return cudaGetLastError();
+}
+
+mp_status assign_impl(const mp_index* idx, const void* K, int32_t n, int32_t* out, cudaStream_t st) {
+  const mp_config& c = idx->cfg;
+  if (n == 0) return MP_OK;
+  const int units = c.batch * c.kv_heads;
+  BlockJob b = make_job(idx);
+  b.srcK = K;
+  b.src_unit_rows = n;
+  b.src_row0 = 0;
+  b.blk0 = 0;
+  b.n_total = n;
+  b.assign = out;
+  b.max_tokens = n;
+  const int nb = (n + c.block_tokens - 1) / c.block_tokens;
+  cudaError_t e = cudaErrorInvalidValue;
+  if (c.dtype == MP_BF16) {
+    if (c.head_dim == 128) e = run_assign<__nv_bfloat16, 128>(b, nb, units, st);
+    else if (c.head_dim == 64) e = run_assign<__nv_bfloat16, 64>(b, nb, units, st);
+  } else {
+    if (c.head_dim == 128) e = run_assign<float, 128>(b, nb, units, st);
+    else if (c.head_dim == 64) e = run_assign<float, 64>(b, nb, units, st);
+  }
+  return e == cudaSuccess ? MP_OK : MP_ECUDA;
 }
 
 template <typename T, int D>

@@ -180,6 +180,17 @@ mp_status mp_cluster_build(mp_index* idx, const void* K, const void* V, int32_t 
 mp_status mp_cluster_update(mp_index* idx, const void* K_new, const void* V_new, int32_t n_new,
                             int32_t* reclustered, void* stream);
 
+/* One Lloyd assignment step against the index's current centroids (pages:
+ * abstract, k-means clustering of the keys; atlas.scime summary, "Approach").
+ * K: [B, H, n, d] device keys in dtype, the keys the index clusters, in token
+ * order, with n == n_clustered (MP_EINVAL otherwise).  For every token t of
+ * block j, assign_out[b, h, t] (device int32 [B, H, n], caller-owned) receives
+ * the slot j * slots_per_block + c of its nearest centroid among the block's
+ * ceil(L_j / T) centroids: argmin_c (|Kc_c|^2 - 2 k_t . Kc_c) in fp32, ties to
+ * the lower slot; for bf16 the dot products run on the tensor cores with fp32
+ * accumulation.  The index is not modified. */
+mp_status mp_cluster_assign(const mp_index* idx, const void* K, int32_t n, int32_t* assign_out, void* stream);
+
 /* One decode step (pages: abstract; atlas.scime summary, "Approach").
  * Q, O: [B, Hq, d].  Per KV head: score every non-empty cluster,
  * s[g,c] = scale * q_g . Kc_c, group score max_g s[g,c]; select clusters in

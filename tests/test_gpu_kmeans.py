@@ -18,18 +18,26 @@ from oracle import multipole as mp
 pytestmark = pytest.mark.gpu
 
 
-def tie_band(X, cents, d_terms=None):
+# Unit roundoff of one fp32 accumulation step of the tensor cores (bf16 keys).
+# Their fp32 adds are not specified as round-to-nearest; a step that truncates
+# errs by up to 2^-23, and the bound takes a further factor of 2 for the
+# alignment of the products inside one MMA.
+U_TC = 2.0 ** -22
+
+
+def tie_band(X, cents, d_terms=None, u_dot=2.0 ** -24):
     """Per-row fp32 error bound of the nearest-centroid decision.
 
     The kernel forms |c|^2 - 2 x.c with d-term fp32 dot products: the error of
-    each distance is at most g (|c|^2 + 2 |x||c|) + u |dist|, g = d u / (1 - d u),
-    u = 2^-24.  The oracle rounds its fp64 distances to fp32 (error u |x - c|^2).
-    A row is a tie if its two nearest centroids are closer than the sum of
-    these bounds for both of them.
+    each distance is at most g (|c|^2 + 2 |x||c|) + u |dist|, g = d u' / (1 - d u'),
+    u = 2^-24 and u' the unit of the dot products' accumulation (u for the
+    fp32 SIMT path, U_TC for the tensor cores).  The oracle rounds its fp64
+    distances to fp32 (error u |x - c|^2).  A row is a tie if its two nearest
+    centroids are closer than the sum of these bounds for both of them.
     """
     u = 2.0 ** -24
     d = X.shape[1] if d_terms is None else d_terms
-    g = d * u / (1 - d * u)
+    g = d * u_dot / (1 - d * u_dot)
     cc = np.sum(cents * cents, axis=1)
     xx = np.sum(X * X, axis=1)
     dist = xx[:, None] + cc[None, :] - 2.0 * (X @ cents.T)
@@ -44,11 +52,22 @@ def tie_band(X, cents, d_terms=None):
     return band
 
 
+def band_for(X, cents):
+    """tie_band of the path that assigns these keys: tensor cores for bf16, fp32 SIMT otherwise."""
+    return tie_band(X, cents, u_dot=U_TC if X.dtype == np.float64 and _is_bf16(X) else 2.0 ** -24)
+
+
+def _is_bf16(X):
+    """True if every value of X is a bf16 number (the keys of a bf16 index)."""
+    x = np.asarray(X, dtype=np.float32)
+    return bool(np.all((x.view(np.uint32) & 0xFFFF) == 0))
+
+
 def first_tie_iteration(hist, X, init):
     """Index of the first Lloyd iteration with a near-tie row (len(hist) if none)."""
     prev = init
     for t, h in enumerate(hist):
-        if np.any(h["gap"] <= tie_band(X, prev)):
+        if np.any(h["gap"] <= band_for(X, prev)):
             return t
         prev = h["cents"]
     return len(hist)
@@ -145,7 +164,7 @@ def compare_trajectories(o, K, V, n, iters, init=None, init_mode="kmeans++"):
                     prev = X[mp.kmeanspp_pick(X, C, mp.stream_uniforms(o["seed"], b * Hk + h, j, 0, C))]
                 else:
                     prev = X[T * np.arange(C)]
-            band = tie_band(X, prev)
+            band = band_for(X, prev)
             assert np.all(hist[k - 1]["gap"][diff] <= band[diff]), \
                 f"block {(b, h, j)} iteration {k}: assignments differ outside the fp32 tie band"
             in_sync[(b, h, j)] = False
@@ -290,3 +309,90 @@ def test_online_update_matches_oracle():
     O_g = g.decode(H.tdev(Q, "f32"), 1 << 20)
     dense = mp.dense_attention(Q, K, V, pos, 2)
     assert np.abs(H.to_np(O_g) - dense).max() <= 1e-4
+
+
+# ----------------------------------------------------------------------------- one assignment step
+def oracle_assign(o, Kc, K, n):
+    """Oracle assignment of every key to its block's centroids: (slots, gap, band) per (b, h)."""
+    Lb, T = o["L_blk"], o["T"]
+    C_blk = -(-Lb // T)
+    out = {}
+    for b in range(o["B"]):
+        for h in range(o["Hkv"]):
+            a_all, gap_all, band_all = [], [], []
+            for j in range(-(-n // Lb)):
+                s0, e0 = j * Lb, min(n, (j + 1) * Lb)
+                C = -(-(e0 - s0) // T)
+                X = K[b, h, s0:e0].astype(np.float64)
+                cents = Kc[b, h, j * C_blk:j * C_blk + C]
+                a, gap = mp.assign_nearest(X, cents)
+                a_all.append(a + j * C_blk)
+                gap_all.append(gap)
+                band_all.append(band_for(X, cents))
+            out[(b, h)] = (np.concatenate(a_all), np.concatenate(gap_all), np.concatenate(band_all))
+    return out
+
+
+@pytest.mark.parametrize("dtype,d,L_blk,T,n", [
+    ("bf16", 128, 8192, 16, 8192 + 3000),     # 512 centroids (two N-halves), then a ragged block of 188
+    ("bf16", 128, 8192, 16, 8192 + 4200),     # ragged block of 263 centroids: a half of 7 centroids
+    ("bf16", 64, 4096, 16, 2 * 4096 + 1000),  # 256 centroids: one half, chunks split over both warp groups
+    ("bf16", 128, 2048, 8, 2048 + 77),        # 256 centroids; a last block of one tile with 10 centroids
+    ("f32", 64, 2048, 16, 2048 + 500),        # fp32 keys: SIMT path
+])
+def test_assign_matches_oracle_except_ties(dtype, d, L_blk, T, n):
+    """One assignment step against the index's own centroids: exact except fp32 ties."""
+    o = H.ocfg(B=1, Hkv=2, Hq=4, d=d, n_max=n, T=T, L_blk=L_blk, dtype=dtype, iters=2, seed=5)
+    K, V, _ = H.cache_for(o, n, comps=200, seed=8)
+    g = gpu_build(o, K, V, n)
+    Kd = H.tdev(K, dtype)
+    a = g.assign(Kd).cpu().numpy().astype(np.int64)
+    torch.cuda.synchronize()
+    assert g.check_device_error() == 0
+    Kc = H.to_np(g.arrays()["Kc"])
+    want = oracle_assign(o, Kc, K, n)
+    for (b, h), (ao, gap, band) in want.items():
+        diff = np.nonzero(a[b, h] != ao)[0]
+        assert np.all(gap[diff] <= band[diff]), f"unit {(b, h)}: {diff.size} rows differ outside the tie band"
+        assert diff.size <= max(2, n // 1000)
+
+
+@pytest.mark.parametrize("d,L_blk,n", [(128, 8192, 8192 + 2100), (64, 4096, 4096 + 600)])
+def test_assign_duplicate_centroids_take_lower_slot(d, L_blk, n):
+    """Bit-identical centroids give bit-identical distances: the lower slot must win.
+
+    Duplicates are placed within one interleaved chain, across chains, across
+    32-column chunks and across the two N-halves of a 512-centroid block; the
+    keys are copies of centroids, so each key's nearest centroid is its own
+    (distance 0) or an exact duplicate of it.
+    """
+    o = H.ocfg(B=1, Hkv=2, Hq=4, d=d, n_max=n, T=16, L_blk=L_blk, dtype="bf16", iters=1, seed=6)
+    K, V, _ = H.cache_for(o, n, comps=100, seed=9)
+    g = gpu_build(o, K, V, n)
+    C_blk = L_blk // 16
+    rng = np.random.default_rng(3)
+    Kc = rng.standard_normal((1, 2, g.slots, d))
+    Kc = np.asarray(torch.from_numpy(Kc).to(torch.bfloat16).float().numpy(), dtype=np.float64)
+    pairs = [(0, 4), (1, 2), (3, 35), (40, 200), (7, 255), (8, 100)]
+    if C_blk == 512:
+        pairs += [(10, 256), (255, 256), (300, 301), (260, 511), (5, 500)]
+    for j in range(-(-n // L_blk)):
+        C = -(-(min(n, (j + 1) * L_blk) - j * L_blk) // 16)
+        for p1, p2 in pairs:
+            if p2 < C:
+                Kc[:, :, j * C_blk + p2] = Kc[:, :, j * C_blk + p1]
+    Kq = np.zeros((1, 2, n, d))
+    for j in range(-(-n // L_blk)):
+        s0, e0 = j * L_blk, min(n, (j + 1) * L_blk)
+        C = -(-(e0 - s0) // 16)
+        pick = rng.integers(0, C, size=e0 - s0)
+        for p1, p2 in pairs:                    # every duplicate pair gets keys
+            if p2 < C:
+                pick[rng.integers(0, e0 - s0, size=4)] = p2
+        Kq[:, :, s0:e0] = Kc[:, :, j * C_blk + pick]
+    arr = g.arrays()
+    arr["Kc"].copy_(H.tdev(Kc, "bf16"))
+    a = g.assign(H.tdev(Kq, "bf16")).cpu().numpy().astype(np.int64)
+    want = oracle_assign(o, Kc, Kq, n)
+    for (b, h), (ao, _, _) in want.items():
+        np.testing.assert_array_equal(a[b, h], ao)

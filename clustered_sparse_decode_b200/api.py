@@ -105,12 +105,16 @@ class MultipoleIndex:
     def decode_phases(self):
         """Names of the intervals between the phase events that decode() records for this index.
 
-        A flat bf16 index with at most 4096 slots per unit decodes with a
-        centroid pass and a value pass (after a reset of its ticket words); the
-        others run a longer kernel pipeline.
+        A flat bf16 index with at most 4096 slots per unit, fewer than 512
+        units and at least 8 tokens decodes with a centroid pass and a value
+        pass (after a reset of its ticket words); the others run a longer
+        kernel pipeline.
         """
         c = self.cfg
-        if c.levels == 1 and c.dtype == "bf16" and self.slots <= 4096:
+        units = c.batch * c.kv_heads
+        if (c.levels == 1 and c.dtype == "bf16" and c.head_dim in (64, 128) and self.slots <= 4096
+                and units < 512 and self.n_tokens >= 8 and c.max_tokens <= (1 << 25)
+                and units * c.max_tokens < 2 ** 31 - 1 and c.q_heads // c.kv_heads in (1, 2, 4, 8)):
             return ["ticket reset", "centroid pass + value pass"]
         if c.levels == 1:
             return ["centroid pass", "select", "token pass", "combine"]

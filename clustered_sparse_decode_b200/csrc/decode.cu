@@ -609,7 +609,7 @@ static DecodeLayout decode_layout(const mp_config& c, int slots, int coarse_slot
 }
 
 size_t stream_scratch_bytes(const mp_config& c, int slots);
-bool stream_supported(const mp_config& c, int slots);
+bool stream_supported(const mp_config& c, int slots, int64_t n_tokens);
 mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
                         size_t scratch_bytes, float scale, cudaStream_t st);
 
@@ -687,7 +687,7 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
                       void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const mp_config& c = idx->cfg;
   // flat bf16 index: the one-kernel streaming path (decode_stream.cu)
-  if (stream_supported(c, idx->slots)) {
+  if (stream_supported(c, idx->slots, idx->n_tokens)) {
     const float sc = prm->scale != 0.f ? prm->scale : 1.0f / sqrtf((float)c.head_dim);
     return stream_decode(idx, Q, O, prm, scratch, scratch_bytes, sc, st);
   }

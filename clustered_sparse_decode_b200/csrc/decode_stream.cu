@@ -61,6 +61,7 @@ constexpr int kMaxGrid = 512;
 struct Args {
   CUtensorMap tmKc;            // Kc as [units*slots rows][D] bf16: 64 x 128 tiles, 128-byte swizzle
   CUtensorMap tmVc;
+  CUtensorMap tmKV;            // Kp and Vp as one map (columns, rows, [half,] key/value): 8-row boxes, 128-byte swizzle
   const __nv_bfloat16* Q;      // [units*G][D]
   __nv_bfloat16* O;            // [units*G][D]
   const __nv_bfloat16* Vc;     // [units][slots][D]
@@ -74,10 +75,10 @@ struct Args {
   int budget, approx;
   int capc;                    // selected-cluster capacity per unit
   float* S;                    // [units][slots][SG] scores (natural units), rows padded to 16 bytes
-  int32_t* tok_src;            // [units][max_tokens] store row of each exact row of the value stream
+  int32_t* boxes;              // [units][max_tokens] packed 8-row boxes of the exact rows (box_pack)
   int32_t* sub_src;            // [units][capc] slot of each selected cluster (subtraction rows)
   float* sub_bias;             // [units][capc] log2 of its size
-  int32_t* hdr;                // [units][2]: exact rows, subtraction rows
+  int32_t* hdr;                // [units][2]: boxes, subtraction rows
   float* pm;                   // [npart][G] partial max (log2 units)
   float* pl;                   // [npart][G] partial normaliser
   float* pacc;                 // [npart][G][D] partial numerator
@@ -98,18 +99,22 @@ struct Geo {
   static constexpr int SLOT = 2 * AREA;                // 1024-byte multiple
   static constexpr int QB = ((G * D * 2 + 127) / 128) * 128;
   static constexpr int OFF_AUX = kNS * SLOT;           // per slot: query rows, cluster offsets, meta
-  static constexpr int AUX = QB + (kRows + 4) * 4 + 32;
+  // centroid pass: query rows, cluster offsets, meta; value pass: meta, biases, row sources
+  static constexpr int AUX_C = QB + (kRows + 4) * 4 + 32;
+  static constexpr int AUX_V = 64 + 2 * kRows * 4;
+  static constexpr int AUX = AUX_C > AUX_V ? AUX_C : AUX_V;
   static constexpr int OFF_UNIT = OFF_AUX + kNS * AUX; // per unit and pass: first partial, number of shares
   static constexpr int OFF_WPRE = OFF_UNIT + kMaxUnits * 16;   // value pass: weight prefix over units
   static constexpr int OFF_HDR = (OFF_WPRE + (kMaxUnits + 1) * 8 + 15) / 16 * 16;   // value pass: stream lengths
   static constexpr int OFF_RED = OFF_HDR + kMaxUnits * 8;
-  static constexpr int OFF_BAR = OFF_RED + 128 * 4;
+  static constexpr int OFF_SRC = OFF_RED + 128 * 4;    // value pass: the producer's ring of 3 chunks' sources
+  static constexpr int OFF_BAR = OFF_SRC + 3 * 2 * kRows * 4;   // (also: kVP producers x 3 x 16 box entries)
   static constexpr int SMEM = OFF_BAR + 2 * kNS * 8 + 16 + 1024;   // + alignment slack
   static_assert(D % 64 == 0, "rows are whole 64-column tiles");
   static_assert(kRows * SG * 4 <= AREA, "subtraction-row scores live in the key area");
   static_assert(AUX % 16 == 0, "16-byte aligned side areas");
   static_assert(OFF_AUX % 1024 == 0 && OFF_UNIT % 16 == 0 && OFF_WPRE % 16 == 0 && OFF_HDR % 16 == 0 &&
-                    OFF_RED % 16 == 0 && OFF_BAR % 16 == 0,
+                    OFF_RED % 16 == 0 && OFF_SRC % 16 == 0 && OFF_BAR % 16 == 0,
                 "regions read with 16-byte vectors and mbarriers need 16-byte alignment");
   static_assert(SMEM <= 232448, "one CTA per SM");
 };
@@ -169,6 +174,22 @@ __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* tm, in
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+// one 8-row box of the key and value stores: a 4-D (d = 128: columns, rows, half,
+// key/value) or 3-D (d = 64: columns, rows, key/value) tensor map, coordinates {0, y, 0[, 0]}
+template <int D>
+__device__ __forceinline__ void tma_box_t(uint32_t dst, const CUtensorMap* tm, int y, uint32_t bar) {
+  if constexpr (D == 128) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %2, %2}], [%4];\n"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(0), "r"(y), "r"(bar)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %2}], [%4];\n"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(0), "r"(y), "r"(bar)
+        : "memory");
+  }
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 // ticket: returns the old value; release orders this CTA's earlier writes (made
@@ -230,6 +251,22 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 // 128-byte swizzle writes to a 1024-byte aligned destination.
 __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)((c >> 3) * kTile + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Box-major chunk layout of the value pass: 16 boxes of 8 rows, box b at
+// b * 32 D bytes holding its key rows, then its value rows, each as D/64
+// 1024-byte atoms [8 rows][128 bytes] (one per 64 columns, 128-byte swizzle):
+// the layout one TMA load of an 8-row box of both the key and the value store
+// writes.  Offset of 16-byte chunk c of row r from the key (or value) part.
+template <int D>
+__device__ __forceinline__ uint32_t bswz(int r, int c) {
+  return (r >> 3) * (32 * D) + (c >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+// offset of chunk c of row r in the layout of the pass (BOX: the value pass's boxes)
+template <bool BOX, int D>
+__device__ __forceinline__ uint32_t lay(int r, int c) {
+  if constexpr (BOX) return bswz<D>(r, c);
+  else return swz(r, c);
 }
 
 // ---------------------------------------------------------------------------
@@ -296,6 +333,7 @@ struct WarpSoftmax {
   }
   // raw dot products q_g . k for the 16 rows of a tile (S = Q K^T with the heads as M rows;
   // this lane: head lane/4, rows 2*(lane%4) + {0,1} + 8*nt)
+  template <bool BOX = false>
   __device__ __forceinline__ void qk(uint32_t kb, int r16, int lane, float (&z)[2][2]) const {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -303,7 +341,7 @@ struct WarpSoftmax {
 #pragma unroll
       for (int kc = 0; kc < D / 32; ++kc) {
         uint32_t b0, b1, b2, b3;
-        ldsm4(kb + swz(r16 + nt * 8 + (lane & 7), 4 * kc + (lane >> 3)), b0, b1, b2, b3);
+        ldsm4(kb + lay<BOX, D>(r16 + nt * 8 + (lane & 7), 4 * kc + (lane >> 3)), b0, b1, b2, b3);
         mma16816(c0, c1, qa[2 * kc][0], qa[2 * kc][1], b0, b1);
         mma16816(e0, e1, qa[2 * kc + 1][0], qa[2 * kc + 1][1], b2, b3);
       }
@@ -315,6 +353,7 @@ struct WarpSoftmax {
   // the state.  P.V is computed as O^T += V^T P^T: the value rows' transpose is
   // the A operand (m-tiles of 16 columns), and the probabilities, already in
   // the B-operand layout, enter as a bf16 hi + lo pair.
+  template <bool BOX = false>
   __device__ __forceinline__ void update(uint32_t vb, int r16, int lane, float (&z)[2][2], float sign) {
     float mx = fmaxf(fmaxf(z[0][0], z[0][1]), fmaxf(z[1][0], z[1][1]));
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
@@ -348,7 +387,7 @@ struct WarpSoftmax {
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
       uint32_t v0, v1, v2, v3;
-      ldsm4t(vb + swz(r16 + (lane & 7) + 8 * (lane >> 4), 2 * mt + ((lane >> 3) & 1)), v0, v1, v2, v3);
+      ldsm4t(vb + lay<BOX, D>(r16 + (lane & 7) + 8 * (lane >> 4), 2 * mt + ((lane >> 3) & 1)), v0, v1, v2, v3);
       mma16816_full(acc[mt], v0, v1, v2, v3, h0, h1);
       mma16816_full(acc[mt], v0, v1, v2, v3, l0, l1);
     }
@@ -491,6 +530,28 @@ __device__ __forceinline__ void cscan2(int a, int b, int& ea, int& eb, int& ta, 
 // weight from the top crosses the budget, and the interval narrows to it.
 // hist: 256 ints of shared memory.
 // ---------------------------------------------------------------------------
+// An 8-row box of the store, packed: first row g (25 bits), valid rows [lo, hi)
+// of the box (lo: 3 bits, hi - 1: 3 bits).  Box b of the run [st, st + cnt):
+// rows st + 8b .. + 7, except a partial last box, which ends at the run's end
+// (its first 8 - cnt % 8 rows repeat the previous box, or belong to the rows
+// before the run, and are not valid); a run of fewer than 8 rows that starts
+// within the first 8 rows takes rows 0..7 instead.  No box reaches past the
+// run's end unless the run lies in rows 0..7, so with at least 8 rows held no
+// box reads a row that was never written.
+__device__ __forceinline__ int32_t box_entry(int st, int cnt, int b) {
+  const int nb = (cnt + 7) >> 3, rem = cnt & 7;
+  int g = st + 8 * b, lo = 0, hi = 8;
+  if (b == nb - 1 && rem) {
+    g = st + cnt - 8;
+    lo = 8 - rem;
+    if (g < 0) { g = 0; lo = st; hi = st + rem; }
+  }
+  return g | (lo << 25) | ((hi - 1) << 28);
+}
+__device__ __forceinline__ int box_row(int32_t e) { return e & ((1 << 25) - 1); }
+__device__ __forceinline__ int box_lo(int32_t e) { return (e >> 25) & 7; }
+__device__ __forceinline__ int box_hi(int32_t e) { return ((e >> 28) & 7) + 1; }
+
 template <int G, int SG>
 __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -616,7 +677,7 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   int tie_before, e2, t1, t2;
   cscan2(tw, 0, tie_before, e2, t1, t2, red);
   uint32_t selbits = 0u;
-  int ntok = 0, nsel = 0;
+  int nsel = 0;
 #pragma unroll
   for (int k = 0; k < kMaxSpt; ++k) {
     if (w[k] > 0) {
@@ -626,51 +687,45 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
         if (key[k] > tau) s = true;
         else if (key[k] == tau) { s = tie_before < need; tie_before += w[k]; }
       }
-      if (s) { selbits |= 1u << k; ntok += w[k]; ++nsel; }
+      if (s) { selbits |= 1u << k; ++nsel; }
     }
   }
-  int tok_base, sub_base, tok_total, sel_total;
-  cscan2(ntok, nsel, tok_base, sub_base, tok_total, sel_total, red);
+  // the exact rows as 8-row boxes of the store: per selected cluster (slot order), then the tail
+  int nbx = 0;
+#pragma unroll
+  for (int k = 0; k < kMaxSpt; ++k)
+    if ((selbits >> k) & 1u) nbx += (w[k] + 7) >> 3;
+  int box_base, sub_base, box_total, sel_total;
+  cscan2(nbx, nsel, box_base, sub_base, box_total, sel_total, red);
 
-  int32_t* tsrc = a.tok_src + (size_t)u * a.max_tokens;
+  int32_t* bx = a.boxes + (size_t)u * a.max_tokens;
   int32_t* ssrc = a.sub_src + (size_t)u * a.capc;
   float* sbias = a.sub_bias + (size_t)u * a.capc;
-  // this thread's selected clusters: mask, subtraction rows and their tokens.  One
-  // compact loop (no unrolled copies of the store code): each warp walks its
-  // lanes' selected clusters one at a time and stores each run coalesced.
-  uint32_t selrem = selbits;
   if (a.sel_mask_out) {
     for (int k = 0; k < spt; ++k)
       if (s0 + k < slots) a.sel_mask_out[(size_t)u * slots + s0 + k] = (selbits >> k) & 1u;
   }
-  int my_base = tok_base;
+  // one compact loop over this thread's selected clusters (offsets re-read: L1 hits)
+  uint32_t selrem = selbits;
 #pragma unroll 1
-  for (;;) {
-    // next selected cluster of this lane (if any), in slot order
-    int k = selrem ? __ffs(selrem) - 1 : -1;
-    int cnt = 0, st = 0;
-    if (k >= 0) {
-      selrem &= selrem - 1;
-      st = __ldg(offu + s0 + k);
-      cnt = __ldg(offu + s0 + k + 1) - st;
+  while (selrem) {
+    const int k = __ffs(selrem) - 1;
+    selrem &= selrem - 1;
+    const int st = __ldg(offu + s0 + k), cnt = __ldg(offu + s0 + k + 1) - st;
+    const int nb = (cnt + 7) >> 3;
+#pragma unroll 1
+    for (int b = 0; b < nb; ++b) bx[box_base + b] = box_entry(st, cnt, b);
+    box_base += nb;
+    if (a.approx) {
       ssrc[sub_base] = s0 + k;
       sbias[sub_base] = log2f((float)cnt);
       ++sub_base;
     }
-    unsigned m = __ballot_sync(kFull, k >= 0);
-    if (!m) break;
-#pragma unroll 1
-    while (m) {
-      const int L = __ffs(m) - 1;
-      m &= m - 1;
-      const int sL = __shfl_sync(kFull, st, L), cL = __shfl_sync(kFull, cnt, L), bL = __shfl_sync(kFull, my_base, L);
-      for (int i = lane; i < cL; i += kWarp) tsrc[bL + i] = sL + i;
-    }
-    my_base += cnt;
   }
-  for (int i = tid; i < a.n_tail; i += kCT) tsrc[tok_total + i] = a.n_clustered + i;
+  const int nbt = (a.n_tail + 7) >> 3;
+  for (int b = tid; b < nbt; b += kCT) bx[box_total + b] = box_entry(a.n_clustered, a.n_tail, b);
   if (tid == 0) {
-    a.hdr[2 * u] = tok_total + a.n_tail;
+    a.hdr[2 * u] = box_total + nbt;
     a.hdr[2 * u + 1] = a.approx ? sel_total : 0;
   }
 }
@@ -817,27 +872,43 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
 }
 
 // ---------------------------------------------------------------------------
-// Value pass: grid CTAs of kCT threads, every warp its own copy pipeline
+// Value pass: grid CTAs of kCT compute threads + one producer warp
 // ---------------------------------------------------------------------------
 // Stream of unit u in weight units: 1 (a placeholder, so that every unit is in
-// exactly one share even when it has no rows), 2 per exact row, 1 per
-// subtraction row.  A row belongs to the share that holds its first weight.
+// exactly one share even when it has no rows), kWB per 8-row box of exact rows,
+// 1 per subtraction row.  A box or row belongs to the share that holds its first
+// weight.  A chunk is up to kBoxes boxes, or up to kRows subtraction rows, of one unit.
+constexpr int kWB = 16;
+constexpr int kBoxes = kRows / 8;
+// Producer warps of the value pass: one per ring slot.  Producer p fills chunks
+// k = p (mod kVP), all in slot p, and so waits on the phases of slot p's empty
+// barrier in order; with more producers than slots a producer could test the
+// parity of a phase two completions ahead of the slot and pass its wait early.
+constexpr int kVP = kNS;
+static_assert(kVP <= kNS, "a producer's empty-barrier waits stay in phase order");
+
 struct VChunk {
-  int unit, kind, p0, cnt;     // kind 0 exact rows, 1 subtraction rows, 2 empty (unit placeholder)
-  int first, last, seg, pad;   // first / last chunk of this CTA's share of the unit; share index
+  int unit, kind, p0, cnt;     // kind 0 boxes, 1 subtraction rows, 2 empty (unit placeholder), 3 end of the share
+  int first, last, seg, valid; // first / last chunk of this CTA's share of the unit; share index; 0: past the share
 };
 
-// Cursor over this CTA's share of the concatenated streams (the same on every warp).
-struct VCursor {
-  long long pos, hi;           // weight position in [lo, hi)
-  int u;                       // unit of pos
-  bool started;                // a chunk of the current unit was already returned
+
+// What the producer tells the compute warps about the chunk in a slot (side area:
+// this, then kRows biases, then kRows row sources).
+struct VMeta {
+  int unit, kind, cnt, flags;  // cnt: boxes loaded (an even number) or subtraction rows; flags 1 first, 2 last
+  int seg, pad0, pad1, pad2;
+  uint8_t lo[kBoxes], hi[kBoxes];   // valid rows [lo, hi) of each box
 };
+constexpr int kVMetaBytes = 64;
+static_assert(sizeof(VMeta) <= kVMetaBytes, "value-pass meta");
 
 template <int D, int G>
-__global__ void __launch_bounds__(kCT, 1) value_pass(const __grid_constant__ Args a) {
+__global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_constant__ Args a) {
   using Gm = Geo<D, G>;
   constexpr int SG = Gm::SG;
+  constexpr int kBoxB = 32 * D;        // one 8-row box: key rows, then value rows
+  static_assert(kBoxes * kBoxB == Gm::SLOT, "a slot holds kBoxes boxes");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -846,222 +917,279 @@ __global__ void __launch_bounds__(kCT, 1) value_pass(const __grid_constant__ Arg
   int* cnsh = cfirst + kMaxUnits;                                               // centroid shares per unit
   int* vfirst = cnsh + kMaxUnits;                                               // value partial base per unit
   int* vnsh = vfirst + kMaxUnits;                                               // value shares per unit
-  int* lens = reinterpret_cast<int*>(smem + Gm::OFF_HDR);                       // [units][2]: exact / subtraction rows
+  int* lens = reinterpret_cast<int*>(smem + Gm::OFF_HDR);                       // [units][2]: boxes / subtraction rows
   int* red = reinterpret_cast<int*>(smem + Gm::OFF_RED);
+  const uint32_t full0 = sb + Gm::OFF_BAR, empty0 = full0 + kNS * 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hq = lane >> 2;
   const int c = blockIdx.x, grid = gridDim.x;
   const float qk2 = a.scale * kLog2e;
+  const long long t_start = gtimer();
+  auto side = [&](int slot) { return smem + Gm::OFF_AUX + slot * Gm::AUX; };
 
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(full0 + 8 * i, kWarp + 1);   // the producer lanes' copy-tracking arrivals + lane 0's (+ TMA bytes)
+      mbar_init(empty0 + 8 * i, kCW);        // one arrival per compute warp
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
   // everything below reads what the centroid pass wrote
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  // per-unit weights and their prefix
-  long long* wtmp = reinterpret_cast<long long*>(smem);   // the first slot is not in use yet
-  for (int u = threadIdx.x; u <= a.units; u += kCT) {
-    const int nt = u < a.units ? __ldcg(a.hdr + 2 * u) : 0, ns = u < a.units ? __ldcg(a.hdr + 2 * u + 1) : 0;
-    if (u < a.units) { lens[2 * u] = nt; lens[2 * u + 1] = ns; }
-    wtmp[u] = u < a.units ? 1 + 2LL * nt + ns : 0LL;
-  }
-  cbar();
-  scan_units<long long>(wtmp, wpre, a.units + 1, 0LL, reinterpret_cast<long long*>(red + 64));
-  const long long WT = wpre[a.units];
-  unit_tables(a, grid, cfirst, cnsh, wpre, vfirst, vnsh, kCT);
-  cbar();
-  scan_units<int>(cnsh, cfirst, a.units, 0, red + 64);
-  scan_units<int>(vnsh, vfirst, a.units, 0, red + 64);
-  for (int u = threadIdx.x; u < a.units; u += kCT) vfirst[u] = a.part_v + vfirst[u] * kCW;
-  cbar();
-
-  const long long lo = share_lo(c, WT, grid), hi = share_lo(c + 1, WT, grid);
-  // the unit holding lo
-  int u0 = 0;
-  {
-    int l = 0, h = a.units - 1;
-    while (l < h) { const int mid = (l + h + 1) >> 1; if (wpre[mid] <= lo) l = mid; else h = mid - 1; }
-    u0 = l;
-  }
-  VCursor cur{lo, hi, u0, false};
-  // next chunk of the share: rows of one unit and one kind, at most kRows
-  auto next = [&](VChunk& ch) -> bool {
-    while (cur.pos < cur.hi && cur.u < a.units) {
-      const int u = cur.u;
-      const long long ub = wpre[u], ue = wpre[u + 1];
-      const int n_tok = lens[2 * u], n_sub = lens[2 * u + 1];
-      const long long rel = cur.pos - ub, rel_end = (cur.hi < ue ? cur.hi : ue) - ub;
-      ch.unit = u;
-      ch.seg = share_index(c, ub, WT, grid);
-      ch.first = !cur.started;
-      // exact rows r with 1 + 2r in [rel, rel_end)
-      const long long t_lo = rel <= 1 ? 0 : (rel - 1 + 1) / 2, t_hi = rel_end <= 1 ? 0 : (rel_end - 1 + 1) / 2;
-      const long long tl = min((long long)n_tok, t_lo), th = min((long long)n_tok, t_hi);
-      const long long s_lo = max(0LL, rel - 1 - 2LL * n_tok), s_hi = max(0LL, rel_end - 1 - 2LL * n_tok);
-      const long long sl = min((long long)n_sub, s_lo), sh = min((long long)n_sub, s_hi);
-      if (tl < th) {
-        ch.kind = 0; ch.p0 = (int)tl; ch.cnt = (int)min((long long)kRows, th - tl);
-        cur.pos = ub + 1 + 2LL * (tl + ch.cnt);                       // first weight after the chunk's rows
-        if (cur.pos > ub + rel_end) cur.pos = ub + rel_end;
-      } else if (sl < sh) {
-        ch.kind = 1; ch.p0 = (int)sl; ch.cnt = (int)min((long long)kRows, sh - sl);
-        cur.pos = ub + 1 + 2LL * n_tok + sl + ch.cnt;
-        if (cur.pos > ub + rel_end) cur.pos = ub + rel_end;
-      } else {
-        // nothing left of this unit in the share (or only its placeholder)
-        ch.kind = 2; ch.p0 = 0; ch.cnt = 0;
-        cur.pos = ub + rel_end;
-      }
-      // is this the last chunk of the share of unit u?
-      bool more = false;
-      if (cur.pos < ub + rel_end) {
-        const long long r2 = cur.pos - ub;
-        const long long t2 = min((long long)n_tok, r2 <= 1 ? 0 : r2 / 2);
-        const long long s2 = min((long long)n_sub, max(0LL, r2 - 1 - 2LL * n_tok));
-        more = t2 < th || s2 < sh;
-      }
-      ch.last = !more;
-      if (!more) {
-        cur.pos = ub + rel_end;
-        cur.u = u + 1;
-        cur.started = false;
-      } else {
-        cur.started = true;
-      }
-      if (ch.kind == 2 && !ch.first) continue;   // a placeholder after rows of the unit adds nothing
-      return true;
+  if (warp < kCW) {
+    // per-unit weights and their prefix; shares per unit
+    long long* wtmp = reinterpret_cast<long long*>(smem);   // the first slot is not in use yet
+    for (int u = threadIdx.x; u <= a.units; u += kCT) {
+      const int nb = u < a.units ? __ldcg(a.hdr + 2 * u) : 0, ns = u < a.units ? __ldcg(a.hdr + 2 * u + 1) : 0;
+      if (u < a.units) { lens[2 * u] = nb; lens[2 * u + 1] = ns; }
+      wtmp[u] = u < a.units ? 1 + (long long)kWB * nb + ns : 0LL;
     }
-    return false;
-  };
+    cbar();
+    scan_units<long long>(wtmp, wpre, a.units + 1, 0LL, reinterpret_cast<long long*>(red + 64));
+    unit_tables(a, grid, cfirst, cnsh, wpre, vfirst, vnsh, kCT);
+    cbar();
+    scan_units<int>(cnsh, cfirst, a.units, 0, red + 64);
+    scan_units<int>(vnsh, vfirst, a.units, 0, red + 64);
+    for (int u = threadIdx.x; u < a.units; u += kCT) vfirst[u] = a.part_v + vfirst[u] * kCW;
+  }
+  __syncthreads();
+  const long long WT = wpre[a.units];
+  const long long lo = share_lo(c, WT, grid), hi = share_lo(c + 1, WT, grid);
 
-  // per-warp copy pipeline: chunk i of the share in slot i % kNS; this warp owns rows [16w, 16w + 16)
+  if (warp >= kCW) {
+    // ======================= producers =======================
+    // kVP warps; chunk k of the share is produced by warp kCW + k % kVP, into slot
+    // k % kNS = k % kVP (its own slot).  Every
+    // producer walks the whole chunk sequence (cheap: the unit's spans are worked
+    // out once per unit) and loads only its own chunks.
+    const int pw = warp - kCW;
+    int u = 0;
+    {
+      int l = 0, h = a.units - 1;
+      while (l < h) { const int mid = (l + h + 1) >> 1; if (wpre[mid] <= lo) l = mid; else h = mid - 1; }
+      u = l;
+    }
+    // this share's part of unit u: boxes [tl, th), subtraction rows [sl, sh), chunks, share index
+    int tl = 0, th = 0, sl = 0, sh = 0, nbc = 0, nch = 0, seg = 0, ci = 0;
+    auto span = [&]() {
+      const long long ub = wpre[u], ue = wpre[u + 1];
+      const int n_box = lens[2 * u], n_sub = lens[2 * u + 1];
+      const long long rel = (lo > ub ? lo : ub) - ub, rel_end = (hi < ue ? hi : ue) - ub;
+      // boxes b with first weight 1 + kWB b in [rel, rel_end); subtraction row s at weight 1 + kWB n_box + s
+      const long long b_lo = rel <= 1 ? 0 : (rel - 1 + kWB - 1) / kWB;
+      const long long b_hi = rel_end <= 1 ? 0 : (rel_end - 1 + kWB - 1) / kWB;
+      tl = (int)min((long long)n_box, b_lo);
+      th = (int)min((long long)n_box, b_hi);
+      const long long sbase = 1 + (long long)kWB * n_box;
+      sl = (int)min((long long)n_sub, max(0LL, rel - sbase));
+      sh = (int)min((long long)n_sub, max(0LL, rel_end - sbase));
+      nbc = (th - tl + kBoxes - 1) / kBoxes;
+      nch = nbc + (sh - sl + kRows - 1) / kRows;
+      if (nch == 0) nch = 1;                       // a share with none of the unit's rows still closes it
+      seg = share_index(c, ub, WT, grid);
+      ci = 0;
+    };
+    const bool any = lo < hi;
+    if (any) span();
+    // chunk descriptor at the cursor, then advance
+    auto next = [&](VChunk& ch) {
+      if (!any || u >= a.units || wpre[u] >= hi) { ch = VChunk{0, 3, 0, 0, 0, 0, 0, 0}; return; }
+      ch.unit = u; ch.seg = seg; ch.first = ci == 0; ch.last = ci == nch - 1; ch.valid = 1;
+      if (ci < nbc) { ch.kind = 0; ch.p0 = tl + ci * kBoxes; ch.cnt = min(kBoxes, th - ch.p0); }
+      else if (tl + nbc * kBoxes < th || sl < sh) {
+        const int j = ci - nbc;
+        ch.kind = 1; ch.p0 = sl + j * kRows; ch.cnt = min(kRows, sh - ch.p0);
+        if (ch.cnt <= 0) { ch.kind = 2; ch.p0 = 0; ch.cnt = 0; }
+      } else { ch.kind = 2; ch.p0 = 0; ch.cnt = 0; }
+      if (++ci == nch) {
+        ++u;
+        if (u < a.units && wpre[u] < hi) span();
+      }
+    };
+    // this warp's chunks k = pw, pw + kVP, ...: box entries copied two own chunks ahead
+    // into a ring of 3 (cp.async, one commit group per own chunk)
+    int* pe = reinterpret_cast<int*>(smem + Gm::OFF_SRC) + pw * 3 * kBoxes;
+    auto prefetch = [&](const VChunk& ch, int e) {
+      if (ch.kind == 0 && lane < ch.cnt)
+        cp4(smem_u32(pe + e * kBoxes + lane), a.boxes + (size_t)ch.unit * a.max_tokens + ch.p0 + lane);
+      cp_commit();
+    };
+    // the next chunk of this warp (skipping the other producers' chunks).  The end
+    // marker (kind 3, index K = the share's chunk count) is published by warp
+    // K % kVP only (k = K); the other producers get k = -1 and stop without
+    // touching the barriers, so that every arrival on a full barrier has landed
+    // before the compute warps that wait on it can exit.
+    int kc = 0;   // index of the chunk the cursor describes next
+    auto next_own = [&](VChunk& ch, int& k) {
+      for (;;) {
+        VChunk t;
+        next(t);
+        const int kk = kc++;
+        if (t.kind == 3) { ch = t; k = kk % kVP == pw ? kk : -1; return; }
+        if (kk % kVP == pw) { ch = t; k = kk; return; }
+      }
+    };
+    VChunk q0, q1, q2;
+    int k0, k1, k2;
+    next_own(q0, k0);
+    prefetch(q0, 0);
+    if (q0.kind != 3) next_own(q1, k1); else { q1 = q0; k1 = k0; }
+    prefetch(q1, 1);
+    for (int i = 0;; ++i) {
+      if (k0 < 0) break;     // the end of the share, published by another producer
+      const int k = k0, slot = k % kNS;
+      const int* es = pe + (i % 3) * kBoxes;
+      cp_wait<1>();          // this lane's copies of the chunk's entries have landed
+      __syncwarp();          // ... and every lane's
+      bool got = true;
+      if (k >= kNS && lane == 0) {
+        while (!(got = mbar_try(empty0 + 8 * slot, ((k / kNS) - 1) & 1))) {
+          if (gtimer() - t_start > a.timeout_ns) { set_error(a.err, E_TIMEOUT); break; }
+        }
+      }
+      if (!__shfl_sync(kFull, got ? 1 : 0, 0)) break;
+      const VChunk ch = q0;
+      unsigned char* sd = side(slot);
+      VMeta* m = reinterpret_cast<VMeta*>(sd);
+      float* sbias = reinterpret_cast<float*>(sd + kVMetaBytes);
+      int* ssrc = reinterpret_cast<int*>(sd + kVMetaBytes + kRows * 4);
+      const uint32_t dst = sb + slot * Gm::SLOT;
+      int nload = 0;                 // boxes loaded: the chunk's, plus a masked copy of the last to an even count
+      int32_t ent = 0;
+      if (ch.kind == 0) {
+        nload = (ch.cnt + 1) & ~1;
+        ent = es[min(lane, ch.cnt - 1)];
+        if ((unsigned)box_row(ent) + 8u > (unsigned)a.max_tokens) set_error(a.err, E_BAD_LIST);
+        if (lane < kBoxes) {
+          m->lo[lane] = lane < ch.cnt ? (uint8_t)box_lo(ent) : (uint8_t)0;
+          m->hi[lane] = lane < ch.cnt ? (uint8_t)box_hi(ent) : (uint8_t)0;
+        }
+      } else if (ch.kind == 1) {
+        // the subtraction rows' slots and biases (one chunk per unit: loaded here)
+        for (int r = lane; r < kRows; r += kWarp) {
+          int src = 0;
+          float bias = 0.f;
+          if (r < ch.cnt) {
+            src = __ldcg(a.sub_src + (size_t)ch.unit * a.capc + ch.p0 + r);
+            bias = __ldcg(a.sub_bias + (size_t)ch.unit * a.capc + ch.p0 + r);
+          }
+          if ((unsigned)src >= (unsigned)a.slots) { set_error(a.err, E_BAD_LIST); src = 0; }
+          ssrc[r] = src;
+          sbias[r] = bias;
+        }
+      }
+      if (lane == 0) {
+        m->unit = ch.unit; m->kind = ch.kind; m->cnt = ch.kind == 0 ? nload : ch.cnt;
+        m->flags = (ch.first ? 1 : 0) | (ch.last ? 2 : 0);
+        m->seg = ch.seg;
+        if (nload > 0)
+          asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;\n" ::"r"(full0 + 8 * slot),
+                       "r"((uint32_t)(nload * kBoxB))
+                       : "memory");
+      }
+      __syncwarp();
+      if (ch.kind == 0 && lane < nload) {
+        // box lane: its 8 key rows and 8 value rows, all columns, in one load
+        const int y = ch.unit * (int)a.max_tokens + box_row(ent);
+        tma_box_t<D>(dst + lane * kBoxB, &a.tmKV, y, full0 + 8 * slot);
+      } else if (ch.kind == 1) {
+        // subtraction rows: value centroid rows and score rows; rows up to the 16-row tile end zero-filled
+        const int rows = (ch.cnt + 15) & ~15;
+        const __nv_bfloat16* Vb = a.Vc + (size_t)ch.unit * a.slots * D;
+        const float* Sb = a.S + (size_t)ch.unit * a.slots * SG;
+        constexpr int RPI = 32 / Gm::CPR;
+        const int cc = lane % Gm::CPR;
+        for (int r = lane / Gm::CPR; r < rows; r += RPI) {
+          const bool v = r < ch.cnt;
+          cp16(dst + kBoxB / 2 + bswz<D>(r, cc), Vb + (size_t)(v ? ssrc[r] : 0) * D + cc * 8, v);
+        }
+        for (int t = lane; t < ch.cnt * (SG / 4); t += kWarp) {
+          const int r = t / (SG / 4), c4 = t % (SG / 4);
+          cp16(dst + (r >> 3) * kBoxB + (r & 7) * SG * 4 + c4 * 16, Sb + (size_t)ssrc[r] * SG + c4 * 4, true);
+        }
+      }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(full0 + 8 * slot) : "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full0 + 8 * slot);
+      if (ch.kind == 3) break;
+      // this warp's chunk after next: describe it and prefetch its entries
+      if (q1.kind != 3) next_own(q2, k2); else { q2 = q1; k2 = k1; }
+      prefetch(q2, (i + 2) % 3);
+      q0 = q1; k0 = k1;
+      q1 = q2; k1 = k2;
+    }
+    cp_wait_all();
+    return;
+  }
+
+  // ======================= compute warps =======================
   const int r16 = warp * 16;
   WarpSoftmax<D, G> ws;
   ws.reset();
-  VChunk q[kNS];
-  bool qv[kNS];
-  int qsrc[kNS];
-  float qbias[kNS];
-  int* bc = red + 120;
-  // load the row sources (lanes 0..15) and subtraction biases of a chunk
-  auto load_src = [&](const VChunk& ch, int& src, float& bias) {
-    src = 0;
-    bias = 0.f;
-    const int r = r16 + (lane & 15);
-    if (ch.kind < 2 && lane < 16 && r < ch.cnt) {
-      if (ch.kind == 0) {
-        src = __ldcg(a.tok_src + (size_t)ch.unit * a.max_tokens + ch.p0 + r);
-        if ((unsigned)src >= (unsigned)a.max_tokens) { set_error(a.err, E_BAD_LIST); src = 0; }
-      } else {
-        src = __ldcg(a.sub_src + (size_t)ch.unit * a.capc + ch.p0 + r);
-        bias = __ldcg(a.sub_bias + (size_t)ch.unit * a.capc + ch.p0 + r);
-        if ((unsigned)src >= (unsigned)a.slots) { set_error(a.err, E_BAD_LIST); src = 0; }
-      }
-    }
-  };
-  // copies of this warp's rows of chunk ch into slot s
-  auto copy = [&](const VChunk& ch, int s, int src) {
-    if (ch.kind < 2 && r16 < ch.cnt) {
-      const uint32_t base = sb + s * Gm::SLOT;
-      const bool tok = ch.kind == 0;
-      const size_t ub = (size_t)ch.unit * (tok ? (size_t)a.max_tokens : (size_t)a.slots);
-      const __nv_bfloat16* Kb = a.Kp + ub * D;
-      const __nv_bfloat16* Vb = (tok ? a.Vp : a.Vc) + ub * D;
-      constexpr int RPI = 32 / Gm::CPR;   // rows per warp instruction
-      const int cc = lane % Gm::CPR;
-#pragma unroll
-      for (int k = 0; k < 16 / RPI; ++k) {
-        const int rl = k * RPI + lane / Gm::CPR;     // row within the warp's 16
-        const int rs = __shfl_sync(kFull, src, rl);
-        const int r = r16 + rl;
-        const bool v = r < ch.cnt;
-        const size_t o = (size_t)rs * D + cc * 8;
-        if (tok) cp16(base + swz(r, cc), v ? (const void*)(Kb + o) : (const void*)a.Kp, v);
-        cp16(base + Gm::AREA + swz(r, cc), v ? (const void*)(Vb + o) : (const void*)a.Vp, v);
-      }
-      if (!tok) {
-        // the subtraction rows' scores, SG floats each, in the key area
-        const float* Sb = a.S + (size_t)ch.unit * a.slots * SG;
-        for (int i = lane; i < 16 * (SG / 4); i += kWarp) {
-          const int rl = i / (SG / 4), c4 = i % (SG / 4);
-          const int rs = __shfl_sync(0xffffffffu >> (32 - min(32, 16 * (SG / 4))), src, rl);
-          const int r = r16 + rl;
-          cp16(base + r * SG * 4 + c4 * 16, Sb + (size_t)rs * SG + c4 * 4, r < ch.cnt);
-        }
-      }
-    }
-    cp_commit();
-  };
-
-  // prologue: kNS - 1 chunks in flight
-#pragma unroll
-  for (int i = 0; i < kNS; ++i) {
-    qv[i] = next(q[i]);
-    if (!qv[i]) q[i] = VChunk{0, 2, 0, 0, 0, 0, 0, 0};
-    load_src(q[i], qsrc[i], qbias[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < kNS - 1; ++i) copy(q[i], i, qsrc[i]);
   int unit_q = -1;
-  for (int i = 0; qv[i % kNS]; ++i) {
-    const int s = i % kNS;
-    // the chunk kNS - 1 ahead goes into the slot computed last iteration
-    copy(q[(i + kNS - 1) % kNS], (i + kNS - 1) % kNS, qsrc[(i + kNS - 1) % kNS]);
-    cp_wait<kNS - 1>();
-    __syncwarp();
-    const VChunk ch = q[s];
-    const float bias = qbias[s];
-    if (ch.first) {
-      if (ch.unit != unit_q) {
-        ws.load_q(a.Q + (size_t)ch.unit * G * D, lane);
-        unit_q = ch.unit;
+  int* bc = red + 120;
+  for (int k = 0;; ++k) {
+    const int slot = k % kNS;
+    bool got = true;
+    while (!(got = mbar_try(full0 + 8 * slot, (k / kNS) & 1))) {
+      if (gtimer() - t_start > 2 * a.timeout_ns) { set_error(a.err, E_TIMEOUT); break; }
+    }
+    if (!got) break;
+    const unsigned char* sd = side(slot);
+    const VMeta* m = reinterpret_cast<const VMeta*>(sd);
+    const int kind = m->kind;
+    if (kind == 3) break;
+    const int u = m->unit, cnt = m->cnt, flags = m->flags, seg = m->seg;
+    if (flags & 1) {
+      if (u != unit_q) {
+        ws.load_q(a.Q + (size_t)u * G * D, lane);
+        unit_q = u;
       }
       ws.reset();
     }
-    if (ch.kind < 2 && r16 < ch.cnt) {
-      const uint32_t base = sb + s * Gm::SLOT;
+    const uint32_t base = sb + slot * Gm::SLOT;
+    if (kind == 0 && 2 * warp < cnt) {
       float z[2][2];
-      if (ch.kind == 0) {
-        ws.qk(base, r16, lane, z);
+      ws.template qk<true>(base, r16, lane, z);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt) {
+        const int bxi = 2 * warp + nt;          // rows nt*8 .. +7 of this warp's tile are box bxi
+        const int blo = m->lo[bxi], bhi = m->hi[bxi];
 #pragma unroll
-          for (int ii = 0; ii < 2; ++ii) {
-            const int r = r16 + nt * 8 + 2 * (lane & 3) + ii;
-            z[nt][ii] = (hq < G && r < ch.cnt) ? z[nt][ii] * qk2 : -INFINITY;
-          }
-      } else {
-        const float* Ss = reinterpret_cast<const float*>(smem + s * Gm::SLOT);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int ii = 0; ii < 2; ++ii) {
-            const int rl = nt * 8 + 2 * (lane & 3) + ii;
-            const int r = r16 + rl;
-            const float b = __shfl_sync(kFull, bias, rl);
-            z[nt][ii] = (hq < G && r < ch.cnt) ? Ss[r * SG + hq] * kLog2e + b : -INFINITY;
-          }
+        for (int ii = 0; ii < 2; ++ii) {
+          const int i = 2 * (lane & 3) + ii;
+          z[nt][ii] = (hq < G && i >= blo && i < bhi) ? z[nt][ii] * qk2 : -INFINITY;
+        }
       }
-      ws.update(base + Gm::AREA, r16, lane, z, ch.kind == 0 ? 1.f : -1.f);
+      ws.template update<true>(base + kBoxB / 2, r16, lane, z, 1.f);
+    } else if (kind == 1 && r16 < cnt) {
+      // the score rows of box b sit at the start of its key part
+      const float* Ss = reinterpret_cast<const float*>(smem + slot * Gm::SLOT);
+      const float* eb = reinterpret_cast<const float*>(sd + kVMetaBytes);
+      float z[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int ii = 0; ii < 2; ++ii) {
+          const int r = r16 + nt * 8 + 2 * (lane & 3) + ii;
+          z[nt][ii] = (hq < G && r < cnt) ? Ss[(r >> 3) * (kBoxB / 4) + (r & 7) * SG + hq] * kLog2e + eb[r] : -INFINITY;
+        }
+      ws.template update<true>(base + kBoxB / 2, r16, lane, z, -1.f);
     }
-    __syncwarp();   // this slot is reused for the chunk kNS ahead
-    // refill the descriptor ring: chunk i + kNS takes slot s
-    const bool more = qv[s] ? next(q[s]) : false;
-    const VChunk done = ch;
-    qv[s] = more;
-    if (!more) q[s] = VChunk{0, 2, 0, 0, 0, 0, 0, 0};
-    load_src(q[s], qsrc[s], qbias[s]);
-    if (done.last) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+    if (flags & 2) {
       // end of this CTA's share of the unit: the warps' partials, then the unit's ticket
-      ws.store(a, vfirst[done.unit] + done.seg * kCW + warp, lane);
+      ws.store(a, vfirst[u] + seg * kCW + warp, lane);
       cbar();
-      if (threadIdx.x == 0) bc[0] = ticket(a.ctl + a.units + done.unit);
-      __syncthreads();
-      if (bc[0] == vnsh[done.unit] - 1) {
+      if (threadIdx.x == 0) bc[0] = ticket(a.ctl + a.units + u);
+      cbar();
+      if (bc[0] == vnsh[u] - 1) {
         // last share of the unit: merge all its partials (centroid and value pass) into the output rows
-        const int u = done.unit;
         combine_unit<D, G>(a, u, cfirst[u] * kCW, cnsh[u] * kCW, vfirst[u], vnsh[u] * kCW);
       }
-      __syncthreads();
+      cbar();
     }
   }
-  cp_wait_all();
 }
 
 }  // namespace stream
@@ -1102,11 +1230,16 @@ static StreamLayout stream_layout(const mp_config& c, int slots) {
 
 size_t stream_scratch_bytes(const mp_config& c, int slots) { return stream_layout(c, slots).bytes; }
 
-bool stream_supported(const mp_config& c, int slots) {
+// The index shapes the two-pass kernels take: flat bf16, d 64 or 128, G in {1, 2, 4, 8},
+// at most kMaxSlots slots and fewer than kMaxUnits units, store rows addressable by
+// the tensor maps (int32 row coordinates, 25-bit box rows), and at least 8 tokens
+// held (no 8-row box of the store reaches a row that was never written).
+bool stream_supported(const mp_config& c, int slots, int64_t n_tokens) {
   const int G = c.q_heads / c.kv_heads;
+  const int64_t U = (int64_t)c.batch * c.kv_heads;
   return c.levels == 1 && c.dtype == MP_BF16 && (c.head_dim == 64 || c.head_dim == 128) &&
-         (G == 1 || G == 2 || G == 4 || G == 8) && slots <= stream::kMaxSlots &&
-         c.batch * c.kv_heads < stream::kMaxUnits;
+         (G == 1 || G == 2 || G == 4 || G == 8) && slots <= stream::kMaxSlots && U < stream::kMaxUnits &&
+         c.max_tokens <= (1 << 25) && U * c.max_tokens < (int64_t)INT32_MAX && n_tokens >= 8;
 }
 
 // cuTensorMapEncodeTiled from the driver, resolved once through the runtime
@@ -1123,15 +1256,41 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// rows x D bf16 matrix, tiles of 64 columns x kRows rows, 128-byte swizzle
-static bool encode_rows(CUtensorMap* tm, const void* base, uint64_t rows, int D) {
+// rows x D bf16 matrix, boxes of 64 columns x box_rows rows, 128-byte swizzle
+static bool encode_rows(CUtensorMap* tm, const void* base, uint64_t rows, int D, int box_rows) {
   auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)stream::kRows};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Kp and Vp ([rows][D] bf16 each, Vp after Kp) as one map whose outermost
+// dimension steps from Kp to Vp: an 8-row box (boxDim {64, 8, [2,] 2}) lands as
+// [key/value][64-column half][8 rows][128 bytes], 128-byte swizzle.  The map
+// covers exactly the two stores, so no box reads outside them.
+static bool encode_store_boxes(CUtensorMap* tm, const void* Kp, const void* Vp, uint64_t rows, int D) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  const intptr_t kv = reinterpret_cast<const char*>(Vp) - reinterpret_cast<const char*>(Kp);
+  if (kv < (intptr_t)(rows * D * 2) || (kv & 15) != 0 || kv >= ((intptr_t)1 << 40)) return false;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (D == 128) {
+    cuuint64_t gdim[4] = {64, rows, 2, 2};
+    cuuint64_t gstride[3] = {256, 128, (cuuint64_t)kv};
+    cuuint32_t box[4] = {64, 8, 2, 2};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(Kp), gdim, gstride, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  cuuint64_t gdim[3] = {64, rows, 2};
+  cuuint64_t gstride[2] = {128, (cuuint64_t)kv};
+  cuuint32_t box[3] = {64, 8, 2};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(Kp), gdim, gstride, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1151,7 +1310,7 @@ static cudaError_t launch_stream_t(const stream::Args& a, int grid, cudaStream_t
   // (griddepcontrol.wait) for that grid's completion before reading its results
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(stream::kCT);
+  cfg.blockDim = dim3(stream::kCT + stream::kVP * kWarp);
   cfg.dynamicSmemBytes = Gm::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1190,13 +1349,14 @@ mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_de
   stream::Args a{};
   const void* Kc = ws_ptr(idx, S_KC);
   a.Vc = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_VC));
-  if (!encode_rows(&a.tmKc, Kc, (uint64_t)U * idx->slots, D) ||
-      !encode_rows(&a.tmVc, a.Vc, (uint64_t)U * idx->slots, D))
+  a.Kp = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_KP));
+  a.Vp = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_VP));
+  if (!encode_rows(&a.tmKc, Kc, (uint64_t)U * idx->slots, D, stream::kRows) ||
+      !encode_rows(&a.tmVc, a.Vc, (uint64_t)U * idx->slots, D, stream::kRows) ||
+      !encode_store_boxes(&a.tmKV, a.Kp, a.Vp, (uint64_t)U * c.max_tokens, D))
     return MP_ECUDA;
   a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.O = static_cast<__nv_bfloat16*>(O);
-  a.Kp = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_KP));
-  a.Vp = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_VP));
   a.off = static_cast<const int32_t*>(ws_ptr(idx, S_OFF));
   a.units = U;
   a.slots = idx->slots;
@@ -1211,7 +1371,7 @@ mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_de
   a.approx = (prm->flags & MP_NO_APPROX) == 0;
   a.capc = L.capc;
   a.S = reinterpret_cast<float*>(base + L.o_S);
-  a.tok_src = reinterpret_cast<int32_t*>(base + L.o_tok);
+  a.boxes = reinterpret_cast<int32_t*>(base + L.o_tok);
   a.sub_src = reinterpret_cast<int32_t*>(base + L.o_ssrc);
   a.sub_bias = reinterpret_cast<float*>(base + L.o_sbias);
   a.hdr = reinterpret_cast<int32_t*>(base + L.o_hdr);

@@ -64,6 +64,7 @@ struct Args {
   CUtensorMap tmKV;            // Kp and Vp as one map (columns, rows, [half,] key/value): 8-row boxes, 128-byte swizzle
   const __nv_bfloat16* Q;      // [units*G][D]
   __nv_bfloat16* O;            // [units*G][D]
+  const __nv_bfloat16* Kc;     // [units][slots][D]
   const __nv_bfloat16* Vc;     // [units][slots][D]
   const __nv_bfloat16* Kp;     // [units][max_tokens][D]
   const __nv_bfloat16* Vp;
@@ -191,6 +192,10 @@ __device__ __forceinline__ void tma_box_t(uint32_t dst, const CUtensorMap* tm, i
         : "memory");
   }
 }
+// bring [p, p + bytes) into L2 (bytes: a multiple of 16, p 16-byte aligned)
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  if (bytes) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 // ticket: returns the old value; release orders this CTA's earlier writes (made
 // visible to this thread by the preceding CTA barrier) before the increment,
@@ -309,105 +314,155 @@ __device__ void unit_tables(const Args& a, int grid, int* cfirst, int* cnsh, con
 // ---------------------------------------------------------------------------
 // Per-warp online softmax over 16-row tiles
 // ---------------------------------------------------------------------------
+// The 16 keys of a tile are the M rows of mma.sync m16n8k16 and 8 "columns" of
+// query heads the N columns: S^T = K Q^T.  With G <= 4 the columns 4..7 repeat
+// the heads of columns 0..3, so that every probability exists twice; the lanes
+// holding columns 0..3 pass its bf16 value (hi) and the lanes holding 4..7 the
+// bf16 rounding of the remainder (lo) into P.V, which therefore keeps ~16
+// significant bits of each weight in one mma per 16 value columns (G = 8: the
+// hi and lo parts go through two mma into the same accumulator).  The
+// transpose from the S^T accumulator layout to the B-operand layout of P.V
+// (keys as K) is movmatrix.trans on the packed bf16 pairs.
+//
+// The running max is lazy: a tile whose logits exceed this lane's max by at
+// most 2^8 is folded with the old max (weights up to 256); only otherwise do
+// the lanes of a column agree on a new max and rescale.
+__device__ __forceinline__ uint32_t movtrans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
 template <int D, int G>
 struct WarpSoftmax {
-  uint32_t qa[D / 16][2];      // A fragments of the query heads (rows 0..7), k-steps of 16
-  float acc[D / 16][4];        // numerator O^T: m-tile mt holds [d = 16 mt + lane/4 (+8)][head 2*(lane%4) (+1)]
-  float m, l;                  // running max (log2 units) and normaliser share of head lane/4
+  static constexpr bool DUP = G <= 4;  // columns 4..7 repeat the heads of columns 0..3
+  static constexpr float kLazy = 8.f;  // log2 of the largest weight folded without a new max
+  uint32_t qb[D / 16][2];      // B fragments of Q^T: [k-step][dims +0 | +8], column lane/4
+  float acc[D / 16][4];        // numerator O^T: m-tile mt holds [d = 16 mt + lane/4 (+8)][column 2*(lane%4) (+1)]
+  float m[2], l[2];            // running max (log2 units) and normaliser of this lane's two columns
+
+  // the head of column 2 (lane % 4) + j, or -1 for an unused column
+  __device__ static __forceinline__ int col_head(int lane, int j) {
+    const int col = 2 * (lane & 3) + j;
+    const int h = DUP ? (col & 3) : col;
+    return h < G ? h : -1;
+  }
+  // this lane's columns carry the lo parts (the repeated columns 4..7)
+  __device__ static __forceinline__ bool lo_cols(int lane) { return DUP && (lane & 3) >= 2; }
+  // row of z[i][.] within the warp's 16
+  __device__ static __forceinline__ int zrow(int lane, int i) { return (lane >> 2) + 8 * i; }
 
   __device__ __forceinline__ void reset() {
-    m = -INFINITY;
-    l = 0.f;
+    m[0] = m[1] = -1e30f;
+    l[0] = l[1] = 0.f;
 #pragma unroll
     for (int n = 0; n < D / 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
   }
   template <typename P>
   __device__ __forceinline__ void load_q(const P* q, int lane) {   // q: [G][D] bf16 (global or shared)
-    const int hq = lane >> 2;
+    const int n = lane >> 2;
+    const int h = DUP ? (n & 3) : n;
     const uint32_t* qs = reinterpret_cast<const uint32_t*>(q);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      qa[ks][0] = hq < G ? qs[(hq * D + ks * 16 + 2 * (lane & 3)) >> 1] : 0u;
-      qa[ks][1] = hq < G ? qs[(hq * D + ks * 16 + 8 + 2 * (lane & 3)) >> 1] : 0u;
+      qb[ks][0] = h < G ? qs[(h * D + ks * 16 + 2 * (lane & 3)) >> 1] : 0u;
+      qb[ks][1] = h < G ? qs[(h * D + ks * 16 + 8 + 2 * (lane & 3)) >> 1] : 0u;
     }
   }
-  // raw dot products q_g . k for the 16 rows of a tile (S = Q K^T with the heads as M rows;
-  // this lane: head lane/4, rows 2*(lane%4) + {0,1} + 8*nt)
+  // raw dot products of the tile's 16 keys with the columns: z[i][j] = key zrow(lane, i), column 2 (lane % 4) + j
   template <bool BOX = false>
   __device__ __forceinline__ void qk(uint32_t kb, int r16, int lane, float (&z)[2][2]) const {
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};   // two accumulation chains
+    const int row = r16 + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      float c0 = 0.f, c1 = 0.f, e0 = 0.f, e1 = 0.f;   // two accumulation chains
-#pragma unroll
-      for (int kc = 0; kc < D / 32; ++kc) {
-        uint32_t b0, b1, b2, b3;
-        ldsm4(kb + lay<BOX, D>(r16 + nt * 8 + (lane & 7), 4 * kc + (lane >> 3)), b0, b1, b2, b3);
-        mma16816(c0, c1, qa[2 * kc][0], qa[2 * kc][1], b0, b1);
-        mma16816(e0, e1, qa[2 * kc + 1][0], qa[2 * kc + 1][1], b2, b3);
-      }
-      z[nt][0] = c0 + e0;
-      z[nt][1] = c1 + e1;
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm4(kb + lay<BOX, D>(row, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
+      if (ks & 1) mma16816_full(c1, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+      else mma16816_full(c0, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
     }
+    z[0][0] = c0[0] + c1[0];
+    z[0][1] = c0[1] + c1[1];
+    z[1][0] = c0[2] + c1[2];
+    z[1][1] = c0[3] + c1[3];
   }
   // Fold a tile with logits z (log2 units, -inf = no term) and weight sign into
-  // the state.  P.V is computed as O^T += V^T P^T: the value rows' transpose is
-  // the A operand (m-tiles of 16 columns), and the probabilities, already in
-  // the B-operand layout, enter as a bf16 hi + lo pair.
+  // the state: O^T += V^T P^T, the value rows' transpose as the A operand.
   template <bool BOX = false>
   __device__ __forceinline__ void update(uint32_t vb, int r16, int lane, float (&z)[2][2], float sign) {
-    float mx = fmaxf(fmaxf(z[0][0], z[0][1]), fmaxf(z[1][0], z[1][1]));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-    const float mnew = fmaxf(m, mx);
-    if (!__any_sync(kFull, mnew != -INFINITY)) return;
-    float pr[2][2];
-    float alpha = 1.f;
-    if (mnew == -INFINITY) {
-      pr[0][0] = pr[0][1] = pr[1][0] = pr[1][1] = 0.f;
-    } else {
-      alpha = ex2(m - mnew);
+    const bool need = fmaxf(z[0][0], z[1][0]) > m[0] + kLazy || fmaxf(z[0][1], z[1][1]) > m[1] + kLazy;
+    if (__any_sync(kFull, need)) {
+      float t0 = fmaxf(z[0][0], z[1][0]), t1 = fmaxf(z[0][1], z[1][1]);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int i = 0; i < 2; ++i) pr[nt][i] = sign * ex2(z[nt][i] - mnew);
-    }
-    m = mnew;
-    l = l * alpha + ((pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]));
-    if (__any_sync(kFull, alpha != 1.f)) {
-      // this lane's accumulators belong to heads 2*(lane%4) and 2*(lane%4) + 1
-      const float a0 = __shfl_sync(kFull, alpha, 8 * (lane & 3));
-      const float a1 = __shfl_sync(kFull, alpha, 8 * (lane & 3) + 4);
+      for (int o = 4; o < 32; o <<= 1) {
+        t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o));
+        t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o));
+      }
+      const float n0 = fmaxf(m[0], t0), n1 = fmaxf(m[1], t1);
+      const float a0 = ex2(m[0] - n0), a1 = ex2(m[1] - n1);
+      m[0] = n0;
+      m[1] = n1;
+      l[0] *= a0;
+      l[1] *= a1;
 #pragma unroll
       for (int n = 0; n < D / 16; ++n) { acc[n][0] *= a0; acc[n][1] *= a1; acc[n][2] *= a0; acc[n][3] *= a1; }
     }
-    const uint32_t h0 = pack_bf16(pr[0][0], pr[0][1]);
-    const uint32_t h1 = pack_bf16(pr[1][0], pr[1][1]);
-    const uint32_t l0 = pack_bf16(pr[0][0] - bf16_lo(h0), pr[0][1] - bf16_hi(h0));
-    const uint32_t l1 = pack_bf16(pr[1][0] - bf16_lo(h1), pr[1][1] - bf16_hi(h1));
+    float p[2][2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) p[i][j] = sign * ex2(z[i][j] - m[j]);
+    l[0] += p[0][0] + p[1][0];
+    l[1] += p[0][1] + p[1][1];
+    const uint32_t h0 = pack_bf16(p[0][0], p[0][1]);    // keys 0..7 of the tile (row lane/4)
+    const uint32_t h1 = pack_bf16(p[1][0], p[1][1]);    // keys 8..15
+    const uint32_t l0 = pack_bf16(p[0][0] - bf16_lo(h0), p[0][1] - bf16_hi(h0));
+    const uint32_t l1 = pack_bf16(p[1][0] - bf16_lo(h1), p[1][1] - bf16_hi(h1));
+    uint32_t b0, b1, c0 = 0u, c1 = 0u;
+    if constexpr (DUP) {
+      const bool lo = lo_cols(lane);
+      b0 = movtrans(lo ? l0 : h0);
+      b1 = movtrans(lo ? l1 : h1);
+    } else {
+      b0 = movtrans(h0);
+      b1 = movtrans(h1);
+      c0 = movtrans(l0);
+      c1 = movtrans(l1);
+    }
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
       uint32_t v0, v1, v2, v3;
       ldsm4t(vb + lay<BOX, D>(r16 + (lane & 7) + 8 * (lane >> 4), 2 * mt + ((lane >> 3) & 1)), v0, v1, v2, v3);
-      mma16816_full(acc[mt], v0, v1, v2, v3, h0, h1);
-      mma16816_full(acc[mt], v0, v1, v2, v3, l0, l1);
+      mma16816_full(acc[mt], v0, v1, v2, v3, b0, b1);
+      if constexpr (!DUP) mma16816_full(acc[mt], v0, v1, v2, v3, c0, c1);
     }
   }
   // this warp's state as partial p: max and normaliser per head, numerator per head and column
   __device__ __forceinline__ void store(const Args& a, int p, int lane) const {
-    const int hq = lane >> 2, h0 = 2 * (lane & 3), h1 = h0 + 1, d0 = lane >> 2;
-    float lt = l;
-    lt += __shfl_xor_sync(kFull, lt, 1);
-    lt += __shfl_xor_sync(kFull, lt, 2);
-    if (hq < G && (lane & 3) == 0) {
-      a.pm[(size_t)p * G + hq] = m;
-      a.pl[(size_t)p * G + hq] = lt;
+    float lt0 = l[0], lt1 = l[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      lt0 += __shfl_xor_sync(kFull, lt0, o);
+      lt1 += __shfl_xor_sync(kFull, lt1, o);
     }
-    float* o0 = a.pacc + ((size_t)p * G + h0) * D + d0;
-    float* o1 = a.pacc + ((size_t)p * G + h1) * D + d0;
+    const bool wr = !lo_cols(lane);
+    const int hd0 = col_head(lane, 0), hd1 = col_head(lane, 1), d0 = lane >> 2;
+    if (wr && lane < 4) {
+      if (hd0 >= 0) { a.pm[(size_t)p * G + hd0] = lt0 != 0.f ? m[0] : -INFINITY; a.pl[(size_t)p * G + hd0] = lt0; }
+      if (hd1 >= 0) { a.pm[(size_t)p * G + hd1] = lt1 != 0.f ? m[1] : -INFINITY; a.pl[(size_t)p * G + hd1] = lt1; }
+    }
+    float* o0 = a.pacc + ((size_t)p * G + (hd0 < 0 ? 0 : hd0)) * D + d0;
+    float* o1 = a.pacc + ((size_t)p * G + (hd1 < 0 ? 0 : hd1)) * D + d0;
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
-      if (h0 < G) { o0[16 * mt] = acc[mt][0]; o0[16 * mt + 8] = acc[mt][2]; }
-      if (h1 < G) { o1[16 * mt] = acc[mt][1]; o1[16 * mt + 8] = acc[mt][3]; }
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[e] = acc[mt][e];
+        if constexpr (DUP) v[e] += __shfl_xor_sync(kFull, acc[mt][e], 2);   // + the lo part of the same head
+      }
+      if (wr && hd0 >= 0) { o0[16 * mt] = v[0]; o0[16 * mt + 8] = v[2]; }
+      if (wr && hd1 >= 0) { o1[16 * mt] = v[1]; o1[16 * mt + 8] = v[3]; }
     }
   }
 };
@@ -552,7 +607,7 @@ __device__ __forceinline__ int box_row(int32_t e) { return e & ((1 << 25) - 1); 
 __device__ __forceinline__ int box_lo(int32_t e) { return (e >> 25) & 7; }
 __device__ __forceinline__ int box_hi(int32_t e) { return ((e >> 28) & 7) + 1; }
 
-template <int G, int SG>
+template <int kD, int G, int SG>
 __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int slots = a.slots;
@@ -745,7 +800,7 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
   int* nsh = first + kMaxUnits;
   int* red = reinterpret_cast<int*>(smem + Gm::OFF_RED);
   const uint32_t full0 = sb + Gm::OFF_BAR, empty0 = full0 + kNS * 8;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hq = lane >> 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long NCH = (long long)a.units * a.cpu;
   const int c = blockIdx.x, grid = gridDim.x;
   const long long lo = share_lo(c, NCH, grid), hi = share_lo(c + 1, NCH, grid);
@@ -794,7 +849,6 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
       if (lane == 0) {
         const uint32_t dst = sb + slot * Gm::SLOT;
         if (cnt > 0) {
-          fence_proxy_async();
           const int y = u * a.slots + p0;
           mbar_arrive_tx(full0 + 8 * slot, (uint32_t)((a.approx ? 2 : 1) * Gm::AREA));
 #pragma unroll
@@ -803,6 +857,7 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
 #pragma unroll
             for (int h = 0; h < D / 64; ++h) tma_tile(dst + Gm::AREA + h * kTile, &a.tmVc, 64 * h, y, full0 + 8 * slot);
           }
+
         } else {
           mbar_arrive(full0 + 8 * slot);
         }
@@ -843,17 +898,22 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
       float z[2][2];
       ws.qk(dst, r16, lane, z);
       float* Srow = a.S + ((size_t)u * a.slots + cm.p0) * SG;
+      const bool wr = !WarpSoftmax<D, G>::lo_cols(lane);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int i = 0; i < 2; ++i) {
+        const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
+        const int n = r < cm.cnt ? offs[r + 1] - offs[r] : 0;
+        const float lg = log2f((float)n);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = r16 + nt * 8 + 2 * (lane & 3) + i;
-          const float S = z[nt][i] * a.scale;
-          if (hq < G && r < cm.cnt) Srow[(size_t)r * SG + hq] = S;
-          const int n = r < cm.cnt ? offs[r + 1] - offs[r] : 0;
-          z[nt][i] = (a.approx && n > 0 && hq < G) ? S * kLog2e + log2f((float)n) : -INFINITY;
+        for (int j = 0; j < 2; ++j) {
+          const int h = WarpSoftmax<D, G>::col_head(lane, j);
+          const float S = z[i][j] * a.scale;
+          if (wr && h >= 0 && r < cm.cnt) Srow[(size_t)r * SG + h] = S;
+          z[i][j] = (a.approx && n > 0 && h >= 0) ? S * kLog2e + lg : -INFINITY;
         }
-      ws.update(dst + Gm::AREA, r16, lane, z, 1.f);
+      }
+      // without centroid terms the value rows are not loaded: nothing to fold
+      if (a.approx) ws.update(dst + Gm::AREA, r16, lane, z, 1.f);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
@@ -864,7 +924,7 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
       if (threadIdx.x == 0) bc[0] = ticket(a.ctl + u);
       cbar();
       const int t = bc[0];
-      if (t == nsh[u] - 1) select_unit<G, SG>(a, u, red, reinterpret_cast<int*>(smem + Gm::OFF_WPRE));
+      if (t == nsh[u] - 1) select_unit<D, G, SG>(a, u, red, reinterpret_cast<int*>(smem + Gm::OFF_WPRE));
       cbar();
     }
   }
@@ -920,7 +980,7 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
   int* lens = reinterpret_cast<int*>(smem + Gm::OFF_HDR);                       // [units][2]: boxes / subtraction rows
   int* red = reinterpret_cast<int*>(smem + Gm::OFF_RED);
   const uint32_t full0 = sb + Gm::OFF_BAR, empty0 = full0 + kNS * 8;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hq = lane >> 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x, grid = gridDim.x;
   const float qk2 = a.scale * kLog2e;
   const long long t_start = gtimer();
@@ -1151,14 +1211,13 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
       float z[2][2];
       ws.template qk<true>(base, r16, lane, z);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int bxi = 2 * warp + nt;          // rows nt*8 .. +7 of this warp's tile are box bxi
+      for (int i = 0; i < 2; ++i) {
+        const int bxi = 2 * warp + i;           // rows 8 i .. 8 i + 7 of this warp's tile are box bxi
         const int blo = m->lo[bxi], bhi = m->hi[bxi];
+        const int rb = lane >> 2;               // row within the box
 #pragma unroll
-        for (int ii = 0; ii < 2; ++ii) {
-          const int i = 2 * (lane & 3) + ii;
-          z[nt][ii] = (hq < G && i >= blo && i < bhi) ? z[nt][ii] * qk2 : -INFINITY;
-        }
+        for (int j = 0; j < 2; ++j)
+          z[i][j] = (WarpSoftmax<D, G>::col_head(lane, j) >= 0 && rb >= blo && rb < bhi) ? z[i][j] * qk2 : -INFINITY;
       }
       ws.template update<true>(base + kBoxB / 2, r16, lane, z, 1.f);
     } else if (kind == 1 && r16 < cnt) {
@@ -1167,12 +1226,14 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
       const float* eb = reinterpret_cast<const float*>(sd + kVMetaBytes);
       float z[2][2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int i = 0; i < 2; ++i) {
+        const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
 #pragma unroll
-        for (int ii = 0; ii < 2; ++ii) {
-          const int r = r16 + nt * 8 + 2 * (lane & 3) + ii;
-          z[nt][ii] = (hq < G && r < cnt) ? Ss[(r >> 3) * (kBoxB / 4) + (r & 7) * SG + hq] * kLog2e + eb[r] : -INFINITY;
+        for (int j = 0; j < 2; ++j) {
+          const int h = WarpSoftmax<D, G>::col_head(lane, j);
+          z[i][j] = (h >= 0 && r < cnt) ? Ss[(r >> 3) * (kBoxB / 4) + (r & 7) * SG + h] * kLog2e + eb[r] : -INFINITY;
         }
+      }
       ws.template update<true>(base + kBoxB / 2, r16, lane, z, -1.f);
     }
     __syncwarp();
@@ -1348,6 +1409,7 @@ mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_de
   grid = std::max(1, std::min(grid, stream::kMaxGrid));
   stream::Args a{};
   const void* Kc = ws_ptr(idx, S_KC);
+  a.Kc = static_cast<const __nv_bfloat16*>(Kc);
   a.Vc = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_VC));
   a.Kp = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_KP));
   a.Vp = static_cast<const __nv_bfloat16*>(ws_ptr(idx, S_VP));

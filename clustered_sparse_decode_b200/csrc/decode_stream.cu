@@ -76,6 +76,7 @@ struct Args {
   int budget, approx;
   int capc;                    // selected-cluster capacity per unit
   float* S;                    // [units][slots][SG] scores (natural units), rows padded to 16 bytes
+  float* shat;                 // [units][slots] group score (max over the group's heads) of each slot
   int32_t* boxes;              // [units][max_tokens] packed 8-row boxes of the exact rows (box_pack)
   int32_t* sub_src;            // [units][capc] slot of each selected cluster (subtraction rows)
   float* sub_bias;             // [units][capc] log2 of its size
@@ -614,7 +615,6 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   const int spt = (slots + kCT - 1) / kCT;
   const int s0 = tid * spt;
   const int32_t* offu = a.off + (size_t)u * (slots + 1);
-  const float* Su = a.S + (size_t)u * slots * SG;
 
   uint32_t key[kMaxSpt];
   int w[kMaxSpt];
@@ -622,30 +622,22 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   int wsum = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   // loads in batches of 8 slots, unconditional (clamped) so that they issue back to back
+  const float* Hu = a.shat + (size_t)u * slots;
 #pragma unroll
   for (int k0 = 0; k0 < kMaxSpt; k0 += 8) {
     if (k0 < spt) {
       int o[9];
-      float4 sv[8][SG / 4];
+      float sv[8];
 #pragma unroll
       for (int k = 0; k <= 8; ++k) o[k] = __ldg(offu + min(s0 + k0 + k, slots));
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-#pragma unroll
-        for (int h = 0; h < SG / 4; ++h)
-          sv[k][h] = __ldcg(reinterpret_cast<const float4*>(Su + (size_t)min(s0 + k0 + k, slots - 1) * SG) + h);
+      for (int k = 0; k < 8; ++k) sv[k] = __ldcg(Hu + min(s0 + k0 + k, slots - 1));
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int c = s0 + k0 + k;
         const bool in = k0 + k < spt && c < slots;
         const int cnt = in ? o[k + 1] - o[k] : 0;
-        float sh = -INFINITY;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float4 v4 = sv[k][g >> 2];
-          const float x = (g & 3) == 0 ? v4.x : (g & 3) == 1 ? v4.y : (g & 3) == 2 ? v4.z : v4.w;
-          sh = fmaxf(sh, x);
-        }
+        const float sh = sv[k];
         key[k0 + k] = cnt > 0 ? ordered_key(sh) : 0u;
         w[k0 + k] = cnt > 0 ? cnt : 0;
         st0[k0 + k] = o[k];
@@ -677,19 +669,29 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   // mode 0: none, 1: all non-empty clusters, 2: threshold
   const int mode = (a.budget <= 0 || W == 0) ? 0 : (W <= a.budget ? 1 : 2);
   uint32_t tau = 0u;
-  int need = 0;
+  int need = 0, ntie = 0;
   if (mode == 2) {
+    // Radix descent over the interval [lo, lo + 2^nb) holding all candidates,
+    // 8 bits a level: a 256-bin histogram of weights (and, on the last level,
+    // where bins are single key values, of key counts), then warp 0 finds the
+    // bin where the weight from the top crosses the budget.
     uint32_t lo = kmin;
-    int nb = kmax == kmin ? 0 : 32 - __clz(kmax - kmin);   // the interval [lo, lo + 2^nb) holds all candidates
+    int nb = kmax == kmin ? 0 : 32 - __clz(kmax - kmin);
     int above = 0;                                          // weight of the keys above the interval
+    int* hcnt = hist + 256;
+    ntie = -1;                                              // keys at tau: unknown unless a level ends on single keys
     while (nb > 0) {
       const int sh = max(nb - 8, 0);
-      for (int i = tid; i < 256; i += kCT) hist[i] = 0;
+      for (int i = tid; i < 256; i += kCT) { hist[i] = 0; hcnt[i] = 0; }
       cbar();
       const unsigned long long hi_excl = (unsigned long long)lo + (1ull << nb);
 #pragma unroll
       for (int k = 0; k < kMaxSpt; ++k)
-        if (w[k] > 0 && key[k] >= lo && (unsigned long long)key[k] < hi_excl) atomicAdd(hist + ((key[k] - lo) >> sh), w[k]);
+        if (w[k] > 0 && key[k] >= lo && (unsigned long long)key[k] < hi_excl) {
+          const int bin = (int)((key[k] - lo) >> sh);
+          atomicAdd(hist + bin, w[k]);
+          if (sh == 0) atomicAdd(hcnt + bin, 1);
+        }
       cbar();
       if (warp == 0) {
         // lane l holds bins 8l .. 8l + 7; running weight from the top bin down
@@ -712,11 +714,12 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
         const unsigned m = __ballot_sync(kFull, found >= 0);
         const int src = 31 - __clz(m);   // the highest lane with a crossing bin holds the answer
         const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
-        if (lane == 0) { red[0] = fb; red[1] = fa; }
+        if (lane == 0) { red[0] = fb; red[1] = fa; red[2] = hcnt[fb]; }
       }
       cbar();
       const int b = red[0];
       above = red[1];
+      if (sh == 0) ntie = red[2];     // the bins of this level were single key values
       lo += (uint32_t)b << sh;
       nb = sh;
       cbar();
@@ -729,8 +732,10 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
 #pragma unroll
     for (int k = 0; k < kMaxSpt; ++k) tw += (key[k] == tau && w[k] > 0) ? w[k] : 0;
   }
-  int tie_before, e2, t1, t2;
-  cscan2(tw, 0, tie_before, e2, t1, t2, red);
+  // the crossing cluster is taken whole; only several clusters at exactly tau
+  // need their order (slot order: an exclusive scan of their weights)
+  int tie_before = 0, e2, t1, t2;
+  if (mode == 2 && ntie != 1) cscan2(tw, 0, tie_before, e2, t1, t2, red);
   uint32_t selbits = 0u;
   int nsel = 0;
 #pragma unroll
@@ -904,13 +909,19 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
         const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
         const int n = r < cm.cnt ? offs[r + 1] - offs[r] : 0;
         const float lg = log2f((float)n);
+        float gmax = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int h = WarpSoftmax<D, G>::col_head(lane, j);
           const float S = z[i][j] * a.scale;
           if (wr && h >= 0 && r < cm.cnt) Srow[(size_t)r * SG + h] = S;
+          if (wr && h >= 0) gmax = fmaxf(gmax, S);
           z[i][j] = (a.approx && n > 0 && h >= 0) ? S * kLog2e + lg : -INFINITY;
         }
+        // the group score of the row: max over the four lanes holding its columns
+        gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 1));
+        gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 2));
+        if ((lane & 3) == 0 && r < cm.cnt) a.shat[(size_t)u * a.slots + cm.p0 + r] = gmax;
       }
       // without centroid terms the value rows are not loaded: nothing to fold
       if (a.approx) ws.update(dst + Gm::AREA, r16, lane, z, 1.f);
@@ -1262,7 +1273,7 @@ static inline size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct StreamLayout {
   int capc, SG, npart;
-  size_t o_S, o_tok, o_ssrc, o_sbias, o_hdr, o_pm, o_pl, o_pacc, o_ctl, ctl_bytes, bytes;
+  size_t o_S, o_shat, o_tok, o_ssrc, o_sbias, o_hdr, o_pm, o_pl, o_pacc, o_ctl, ctl_bytes, bytes;
 };
 
 static StreamLayout stream_layout(const mp_config& c, int slots) {
@@ -1275,6 +1286,7 @@ static StreamLayout stream_layout(const mp_config& c, int slots) {
   L.capc = ((slots + 3) & ~3) + 64;
   size_t cur = 0;
   L.o_S = cur; cur = a256(cur + U * slots * L.SG * 4);
+  L.o_shat = cur; cur = a256(cur + U * slots * 4);
   L.o_tok = cur; cur = a256(cur + U * (size_t)c.max_tokens * 4);
   L.o_ssrc = cur; cur = a256(cur + U * L.capc * 4);
   L.o_sbias = cur; cur = a256(cur + U * L.capc * 4);
@@ -1433,6 +1445,7 @@ mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_de
   a.approx = (prm->flags & MP_NO_APPROX) == 0;
   a.capc = L.capc;
   a.S = reinterpret_cast<float*>(base + L.o_S);
+  a.shat = reinterpret_cast<float*>(base + L.o_shat);
   a.boxes = reinterpret_cast<int32_t*>(base + L.o_tok);
   a.sub_src = reinterpret_cast<int32_t*>(base + L.o_ssrc);
   a.sub_bias = reinterpret_cast<float*>(base + L.o_sbias);

@@ -85,7 +85,8 @@ struct Args {
   float* pl;                   // [npart][G] partial normaliser
   float* pacc;                 // [npart][G][D] partial numerator
   int part_v;                  // first partial of the value pass (the centroid pass uses [0, part_v));
-                               // per (unit, share, warp): (first[u] + share index) * kCW + warp
+                               // per (unit u, share c, warp): (c + u) * kCW + warp (unique: shares are
+                               // contiguous, so the overlapping (c, u) pairs form a staircase)
   int32_t* ctl;                // [u] centroid tickets; [U + u] value tickets
   uint8_t* sel_mask_out;       // optional [units][slots]
   float* scores_out;           // optional [units][slots]
@@ -300,16 +301,10 @@ __device__ __forceinline__ int shares_of(long long xb, long long xe, long long N
 __device__ __forceinline__ int share_index(int c, long long xb, long long N, int grid) {
   return shares_nonempty(share_owner(xb, N, grid), c, N, grid);
 }
-// Per unit: number of shares (partials of share s: (first + s) * kCW + warp) of the centroid pass (chunks [u * cpu, (u + 1) * cpu) of units * cpu) and, if
-// wpre is given, of the value pass (weights [wpre[u], wpre[u + 1]) of wpre[units]).
-__device__ void unit_tables(const Args& a, int grid, int* cfirst, int* cnsh, const long long* wpre, int* vfirst,
-                            int* vnsh, int nthreads) {
-  const long long NCH = (long long)a.units * a.cpu;
-  for (int u = threadIdx.x; u < a.units; u += nthreads) {
-    cnsh[u] = shares_of((long long)u * a.cpu, (long long)(u + 1) * a.cpu, NCH, grid);
-    if (wpre) vnsh[u] = shares_of(wpre[u], wpre[u + 1], wpre[a.units], grid);
-  }
-  __syncwarp();
+// the s-th of the shares holding positions from xb on (with N >= grid every
+// share is non-empty; with N < grid every non-empty share holds one position)
+__device__ __forceinline__ int nth_share(int s, long long xb, long long N, int grid) {
+  return N >= grid ? share_owner(xb, N, grid) + s : share_owner(xb + s, N, grid);
 }
 
 // ---------------------------------------------------------------------------
@@ -468,44 +463,77 @@ struct WarpSoftmax {
   }
 };
 
-// Merge the partials [p0, p0 + n0) and [p1, p1 + n1) of unit u into its output
-// rows (compute threads; one thread per 4 columns of a head, online over the partials).
+// Merge all partials of unit u into its output rows: kCW per share of the
+// centroid pass (chunks [u cpu, (u + 1) cpu) of units cpu) and of the value
+// pass (nvs shares from weight position vb of VN), share c's at (c + u) kCW.
+// (compute threads; one thread per 4 columns of a head, online over the partials)
 template <int D, int G>
-__device__ void combine_unit(const Args& a, int u, int p0, int n0, int p1, int n1) {
-  const int n = n0 + n1;
-  for (int e = threadIdx.x; e < G * D / 4; e += kCT) {
+__device__ void combine_unit(const Args& a, int u, int grid, long long vb, int nvs, long long VN) {
+  constexpr int kCB = 8;                    // partials loaded per round
+  const long long CN = (long long)a.units * a.cpu, cb = (long long)u * a.cpu;
+  const int ncs = shares_of(cb, cb + a.cpu, CN, grid);
+  const int n = (ncs + nvs) * kCW;
+  // partial j: share j / kCW of the concatenated lists, warp j % kCW (the
+  // shares of a list are consecutive CTAs unless the list has empty shares)
+  const int cc0 = share_owner(cb, CN, grid), vc0 = share_owner(vb, VN, grid);
+  const bool cseq = CN >= grid, vseq = VN >= grid;
+  auto part = [&](int j) -> size_t {
+    const int sh = j / kCW, w = j % kCW;
+    if (sh < ncs) return (size_t)((cseq ? cc0 + sh : nth_share(sh, cb, CN, grid)) + u) * kCW + w;
+    const int s2 = sh - ncs;
+    return (size_t)a.part_v + (size_t)((vseq ? vc0 + s2 : nth_share(s2, vb, VN, grid)) + u) * kCW + w;
+  };
+  // SPLIT adjacent threads share an output group of 4 columns of a head: each
+  // folds every SPLIT-th partial, then the states merge across the lanes
+  constexpr int NE = G * D / 4;
+  constexpr int SPLIT = NE >= kCT ? 1 : (kCT / NE >= 8 ? 8 : kCT / NE);
+  const int part_i = threadIdx.x % SPLIT;
+  for (int e = threadIdx.x / SPLIT; e < NE; e += kCT / SPLIT) {
     const int g = (e * 4) / D, d = (e * 4) % D;
     float M = -INFINITY, L = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < n; j0 += 16) {
-      float mj[16], lj[16];
-      float4 xj[16];
+    for (int j0 = part_i; j0 < n; j0 += kCB * SPLIT) {
+      float mj[kCB], lj[kCB];
+      float4 xj[kCB];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int jj = min(j0 + k, n - 1);
-        const size_t p = jj < n0 ? p0 + jj : p1 + jj - n0;
-        mj[k] = j0 + k < n ? __ldcg(a.pm + p * G + g) : -INFINITY;
+      for (int k = 0; k < kCB; ++k) {
+        const int j = j0 + k * SPLIT;
+        const size_t p = part(min(j, n - 1));
+        mj[k] = j < n ? __ldcg(a.pm + p * G + g) : -INFINITY;
         lj[k] = __ldcg(a.pl + p * G + g);
         xj[k] = __ldcg(reinterpret_cast<const float4*>(a.pacc + (p * G + g) * D + d));
       }
       float Mn = M;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) Mn = fmaxf(Mn, mj[k]);
+      for (int k = 0; k < kCB; ++k) Mn = fmaxf(Mn, mj[k]);
       if (Mn == -INFINITY) continue;
       const float s0 = M == -INFINITY ? 0.f : ex2(M - Mn);
       o.x *= s0; o.y *= s0; o.z *= s0; o.w *= s0;
       L *= s0;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < kCB; ++k) {
         const float f = mj[k] == -INFINITY ? 0.f : ex2(mj[k] - Mn);
         o.x += f * xj[k].x; o.y += f * xj[k].y; o.z += f * xj[k].z; o.w += f * xj[k].w;
         L += f * lj[k];
       }
       M = Mn;
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat16* out = a.O + ((size_t)u * G + g) * D + d;
-    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16(o.x * inv, o.y * inv), pack_bf16(o.z * inv, o.w * inv));
+#pragma unroll
+    for (int sft = 1; sft < SPLIT; sft <<= 1) {
+      const float M2 = __shfl_xor_sync(kFull, M, sft), L2 = __shfl_xor_sync(kFull, L, sft);
+      const float x2 = __shfl_xor_sync(kFull, o.x, sft), y2 = __shfl_xor_sync(kFull, o.y, sft);
+      const float z2 = __shfl_xor_sync(kFull, o.z, sft), w2 = __shfl_xor_sync(kFull, o.w, sft);
+      const float Mn = fmaxf(M, M2);
+      const float f1 = M == -INFINITY ? 0.f : ex2(M - Mn), f2 = M2 == -INFINITY ? 0.f : ex2(M2 - Mn);
+      o.x = o.x * f1 + x2 * f2; o.y = o.y * f1 + y2 * f2; o.z = o.z * f1 + z2 * f2; o.w = o.w * f1 + w2 * f2;
+      L = L * f1 + L2 * f2;
+      M = Mn;
+    }
+    if (part_i == 0) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat16* out = a.O + ((size_t)u * G + g) * D + d;
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16(o.x * inv, o.y * inv), pack_bf16(o.z * inv, o.w * inv));
+    }
   }
 }
 
@@ -801,8 +829,6 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
   // TMA tiles with 128-byte swizzle need 1024-byte aligned destinations
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
-  int* first = reinterpret_cast<int*>(smem + Gm::OFF_UNIT);
-  int* nsh = first + kMaxUnits;
   int* red = reinterpret_cast<int*>(smem + Gm::OFF_RED);
   const uint32_t full0 = sb + Gm::OFF_BAR, empty0 = full0 + kNS * 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -874,9 +900,6 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
   }
 
   // ======================= compute warps =======================
-  unit_tables(a, grid, first, nsh, nullptr, nullptr, nullptr, kCT);
-  cbar();
-  scan_units<int>(nsh, first, a.units, 0, red + 64);
   WarpSoftmax<D, G> ws;
   ws.reset();
   int* bc = red + 120;
@@ -930,12 +953,13 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
     if (cm.flags & 2) {
       // end of this CTA's share of unit u: the warps' partials, then the unit's ticket
-      ws.store(a, (first[u] + cm.seg) * kCW + warp, lane);
+      ws.store(a, (c + u) * kCW + warp, lane);
       cbar();
       if (threadIdx.x == 0) bc[0] = ticket(a.ctl + u);
       cbar();
       const int t = bc[0];
-      if (t == nsh[u] - 1) select_unit<D, G, SG>(a, u, red, reinterpret_cast<int*>(smem + Gm::OFF_WPRE));
+      if (t == shares_of((long long)u * a.cpu, (long long)(u + 1) * a.cpu, NCH, grid) - 1)
+        select_unit<D, G, SG>(a, u, red, reinterpret_cast<int*>(smem + Gm::OFF_WPRE));
       cbar();
     }
   }
@@ -984,10 +1008,6 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   long long* wpre = reinterpret_cast<long long*>(smem + Gm::OFF_WPRE);          // [units + 1] weight prefix
-  int* cfirst = reinterpret_cast<int*>(smem + Gm::OFF_UNIT);                    // centroid partial base per unit
-  int* cnsh = cfirst + kMaxUnits;                                               // centroid shares per unit
-  int* vfirst = cnsh + kMaxUnits;                                               // value partial base per unit
-  int* vnsh = vfirst + kMaxUnits;                                               // value shares per unit
   int* lens = reinterpret_cast<int*>(smem + Gm::OFF_HDR);                       // [units][2]: boxes / subtraction rows
   int* red = reinterpret_cast<int*>(smem + Gm::OFF_RED);
   const uint32_t full0 = sb + Gm::OFF_BAR, empty0 = full0 + kNS * 8;
@@ -1007,7 +1027,7 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
   // everything below reads what the centroid pass wrote
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   if (warp < kCW) {
-    // per-unit weights and their prefix; shares per unit
+    // per-unit weights and their prefix
     long long* wtmp = reinterpret_cast<long long*>(smem);   // the first slot is not in use yet
     for (int u = threadIdx.x; u <= a.units; u += kCT) {
       const int nb = u < a.units ? __ldcg(a.hdr + 2 * u) : 0, ns = u < a.units ? __ldcg(a.hdr + 2 * u + 1) : 0;
@@ -1016,11 +1036,6 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
     }
     cbar();
     scan_units<long long>(wtmp, wpre, a.units + 1, 0LL, reinterpret_cast<long long*>(red + 64));
-    unit_tables(a, grid, cfirst, cnsh, wpre, vfirst, vnsh, kCT);
-    cbar();
-    scan_units<int>(cnsh, cfirst, a.units, 0, red + 64);
-    scan_units<int>(vnsh, vfirst, a.units, 0, red + 64);
-    for (int u = threadIdx.x; u < a.units; u += kCT) vfirst[u] = a.part_v + vfirst[u] * kCW;
   }
   __syncthreads();
   const long long WT = wpre[a.units];
@@ -1056,7 +1071,7 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
       nbc = (th - tl + kBoxes - 1) / kBoxes;
       nch = nbc + (sh - sl + kRows - 1) / kRows;
       if (nch == 0) nch = 1;                       // a share with none of the unit's rows still closes it
-      seg = share_index(c, ub, WT, grid);
+      seg = 0;
       ci = 0;
     };
     const bool any = lo < hi;
@@ -1209,7 +1224,7 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
     const VMeta* m = reinterpret_cast<const VMeta*>(sd);
     const int kind = m->kind;
     if (kind == 3) break;
-    const int u = m->unit, cnt = m->cnt, flags = m->flags, seg = m->seg;
+    const int u = m->unit, cnt = m->cnt, flags = m->flags;
     if (flags & 1) {
       if (u != unit_q) {
         ws.load_q(a.Q + (size_t)u * G * D, lane);
@@ -1251,13 +1266,14 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
     if (flags & 2) {
       // end of this CTA's share of the unit: the warps' partials, then the unit's ticket
-      ws.store(a, vfirst[u] + seg * kCW + warp, lane);
+      ws.store(a, a.part_v + (c + u) * kCW + warp, lane);
       cbar();
       if (threadIdx.x == 0) bc[0] = ticket(a.ctl + a.units + u);
       cbar();
-      if (bc[0] == vnsh[u] - 1) {
+      const int nvs = shares_of(wpre[u], wpre[u + 1], WT, grid);
+      if (bc[0] == nvs - 1) {
         // last share of the unit: merge all its partials (centroid and value pass) into the output rows
-        combine_unit<D, G>(a, u, cfirst[u] * kCW, cnsh[u] * kCW, vfirst[u], vnsh[u] * kCW);
+        combine_unit<D, G>(a, u, grid, wpre[u], nvs, WT);
       }
       cbar();
     }

@@ -381,6 +381,111 @@ def run_ours(args, w):
     return 0
 
 
+def run_online(args, w):
+    """Online workload: build on the prompt, then per generated token append it
+    (mp_cluster_update: re-clusters the open block every update_interval tokens or
+    at a block end) and decode one step.  Reports decode plus amortised update
+    time per generated token, device-timed (CUDA events around each call, L2
+    flushed between tokens outside the events)."""
+    import torch
+    import torch.distributed as dist
+
+    from clustered_sparse_decode_b200 import Config, MultipoleIndex, synth
+    from clustered_sparse_decode_b200 import build as libbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    libbuild.build()
+    dev = torch.device("cuda", local)
+    B, Hkv, Hq, d, n0, ng = w["B"], w["Hkv"], w["Hq"], w["d"], w["n"], w["n_gen"]
+    if args.gen_tokens > 0:
+        ng = min(ng, args.gen_tokens)
+    tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+    K, V, _ = synth.make_cache(B, Hkv, n0 + ng, d, w["comps"], w["sigma"], radius=w["radius"], outliers=w["outliers"],
+                               dtype=w["dtype"], seed=w["seed"] + 100 * rank, drift=w.get("drift"))
+    Kd = torch.from_numpy(K).to(dev).to(tdt)
+    Vd = torch.from_numpy(V).to(dev).to(tdt)
+    del K, V
+    Kgen = Kd[:, :, n0:].permute(2, 0, 1, 3).contiguous()   # [ng, B, Hkv, d]: token t's rows contiguous
+    Vgen = Vd[:, :, n0:].permute(2, 0, 1, 3).contiguous()
+    cfg = Config(batch=B, kv_heads=Hkv, q_heads=Hq, head_dim=d, max_tokens=n0 + ng, tokens_per_centroid=w["T"],
+                 block_tokens=w["L_blk"], kmeans_iters=w["iters"], update_interval=w["update_interval"],
+                 dtype=w["dtype"], seed=w["seed"])
+    idx = MultipoleIndex(cfg, device=dev)
+    idx.build(Kd[:, :, :n0].contiguous(), Vd[:, :, :n0].contiguous())
+    del Kd, Vd
+    torch.cuda.synchronize()
+    Qh = synth.make_queries(args.warmup + ng, B, Hq, d, w["dtype"], seed=w["seed"] + 7 + 100 * rank)
+    Q = torch.from_numpy(Qh).to(dev).to(tdt)
+    O = torch.empty((B, Hq, d), dtype=tdt, device=dev)
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
+    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for s in range(args.warmup):
+        flush_w.zero_()
+        flush_r.amax()
+        idx.decode(Q[s], w["budget"], out=O)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(ng)]
+    fired = []
+    for t in range(ng):
+        flush_w.zero_()
+        flush_r.amax()
+        e = ev[t]
+        e[0].record(stream)
+        fired.append(idx.update(Kgen[t].unsqueeze(2), Vgen[t].unsqueeze(2)))
+        e[1].record(stream)
+        idx.decode(Q[args.warmup + t], w["budget"], out=O)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if idx.check_device_error() != 0:
+        raise RuntimeError("device error in the online run")
+    upd = [ev[t][0].elapsed_time(ev[t][1]) for t in range(ng)]
+    upd_ms = sum(upd)
+    n_fired = sum(fired)
+    fired_ms = sum(u for u, f in zip(upd, fired) if f)
+    dec_ms = sum(ev[t][1].elapsed_time(ev[t][2]) for t in range(ng))
+    tot_tokens, tot_s = aggregate(B * ng, (upd_ms + dec_ms) / 1e3, dist)
+    us_per_token = 1e6 * tot_s / ng
+    if rank == 0:
+        line = {
+            "metric": "online decode + amortised cluster update, us per generated token", "value": us_per_token,
+            "unit": "us/token", "n_gpus": world, "steps": ng, "warmup": args.warmup,
+            "ms_per_step": us_per_token / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": w["dtype"], "data": "synthetic",
+            "config": {"workload": args.workload, "batch": B, "kv_heads": Hkv, "q_heads": Hq, "head_dim": d,
+                       "prompt": n0, "generated": ng, "budget": w["budget"], "block_tokens": w["L_blk"],
+                       "update_interval": w["update_interval"], "kmeans_iters": w["iters"],
+                       "l2": "flushed before every generated token (2x L2 written, then 2x L2 read)",
+                       "parallelism": f"dp{world} (independent batches)"},
+            "decode_us_per_token": 1e3 * dec_ms / ng, "update_us_per_token": 1e3 * upd_ms / ng,
+            "reclusterings": n_fired, "recluster_ms_each": fired_ms / max(n_fired, 1),
+            "append_us_each": 1e3 * (upd_ms - fired_ms) / max(ng - n_fired, 1), "tokens_per_s": tot_tokens / tot_s,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def assign_flops(w):
     """Algorithmic flops of one assignment step: 2 L_j C_j d per (unit, block), C_j = ceil(L_j / T)."""
     n, Lb, T, d = w["n"], w["L_blk"], w["T"], w["d"]
@@ -456,6 +561,8 @@ def main(argv=None):
     ap.add_argument("--ref-seconds-per-step", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-assign", action="store_true", help="skip the timed k-means assignment step")
+    ap.add_argument("--gen-tokens", type=int, default=0,
+                    help="online workloads: generated tokens to time (0 = all of the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -463,6 +570,8 @@ def main(argv=None):
     w = synth.workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)
+    if "n_gen" in w:
+        return run_online(args, w)
     return run_ours(args, w)
 
 

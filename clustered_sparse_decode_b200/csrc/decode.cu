@@ -657,8 +657,13 @@ static cudaError_t launch_pass_any(int dtype, int D, int G, const PassArgs& a, i
 }
 
 static cudaError_t launch_select(const SelectArgs& a, int units, cudaStream_t st) {
+  // the 48 KB default limit covers static plus dynamic shared memory
+  static size_t static_smem = [] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, select_kernel) == cudaSuccess ? fa.sharedSizeBytes : (size_t)4096;
+  }();
   size_t smem = (size_t)a.shat_cap * 12;
-  if (smem > 48 * 1024) {
+  if (smem + static_smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }

@@ -212,6 +212,163 @@ kmeanspp_kernel(BlockJob b) {
   }
 }
 
+// The same seeding with far fewer key reads (Elkan, "Using the triangle
+// inequality to accelerate k-means", ICML 2003).  Each point keeps its nearest
+// centre a_i besides D_i^2.  When centre k is at least twice D_i away from
+// c_{a_i}, |x_i - c_k| >= |c_k - c_{a_i}| - D_i >= D_i, so D_i cannot drop and
+// row i is not read.  The test carries a relative margin of 1e-9, far above
+// the fp64 rounding of the squared distances (about 130 ulp), so a skipped row
+// is one whose recomputed D^2 would have lost the min: D^2 and the picks equal
+// those of the full pass.  Per pick: centre-to-centre distances (thread per
+// earlier centre), a compacted list of the rows left to recompute (thread per
+// row, 16-byte loads), then the running sum in 32-row chunks per warp.
+constexpr int kPPrThreads = 512;
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& u, float* f);
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4& u, float* f) {
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y); f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// fp64 squared distance of one row (16-byte aligned) to the centre in s_c
+template <typename T, int D, bool NC>
+__device__ __forceinline__ double row_dist2(const T* x, const double* s_c) {
+  constexpr int EPW = 16 / sizeof(T);
+  constexpr int NB = (D / EPW) / 2 < 8 ? (D / EPW) / 2 : 8;   // 16-byte words in flight per thread
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  double acc = 0.0;
+#pragma unroll 1
+  for (int w0 = 0; w0 < D / EPW; w0 += NB) {
+    uint4 u[NB];
+#pragma unroll
+    for (int w = 0; w < NB; ++w) u[w] = NC ? __ldg(xv + w0 + w) : xv[w0 + w];
+#pragma unroll
+    for (int w = 0; w < NB; ++w) {
+      float f[EPW];
+      unpack16<T>(u[w], f);
+#pragma unroll
+      for (int e = 0; e < EPW; ++e) {
+        const double dd = (double)f[e] - s_c[(w0 + w) * EPW + e];
+        acc = fma(dd, dd, acc);
+      }
+    }
+  }
+  return acc;
+}
+
+size_t kmeanspp_pruned_smem(int L_blk, int C_blk) {
+  return (size_t)L_blk * (sizeof(double) + 2 * sizeof(uint16_t)) + (size_t)C_blk * sizeof(double) + 16;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPPrThreads, 2)
+kmeanspp_pruned_kernel(BlockJob b) {
+  constexpr int NT = kPPrThreads, NW = NT / kWarp;
+  extern __shared__ double s_d2[];                                   // [L_blk] D^2
+  double* s_cc = s_d2 + b.L_blk;                                     // [C_blk] |c_k - c_j|^2
+  uint16_t* s_a = reinterpret_cast<uint16_t*>(s_cc + b.C_blk);      // [L_blk] nearest centre
+  uint16_t* s_list = s_a + b.L_blk;                                  // [L_blk] rows to recompute
+  __shared__ double s_c[D];
+  __shared__ double s_w[NW];
+  __shared__ int s_pick, s_n;
+  const BlockGeo g = block_geo(b);
+  if (g.L == 0) return;
+  const int tid = threadIdx.x, lane = tid % kWarp, warp = tid / kWarp;
+  const T* src = reinterpret_cast<const T*>(b.srcK) + src_row(b, g.unit, g.s) * D;
+  T* Kc = reinterpret_cast<T*>(b.Kc) + ((size_t)g.unit * b.slots + (size_t)g.j * b.C_blk) * D;
+  // each warp sums and searches a contiguous range of rows, in chunks of 32
+  const int rpw = ((g.L + NW - 1) / NW + kWarp - 1) / kWarp * kWarp;
+  const int wr0 = min(g.L, warp * rpw), wr1 = min(g.L, wr0 + rpw);
+
+  double u0 = stream_uniform(b.seed, g.unit, g.j, 0, 0);
+  int first = (int)floor(u0 * (double)g.L);
+  first = min(first, g.L - 1);
+  int pick = first;
+  for (int k = 0; k < g.C; ++k) {
+    if (tid < D) {
+      T v = src[(size_t)pick * D + tid];
+      Kc[(size_t)k * D + tid] = v;
+      s_c[tid] = (double)to_f32(v);
+    }
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    // distances from centre k to the earlier centres (rows of Kc written by this CTA)
+#pragma unroll 1
+    for (int j = tid; j < k; j += NT) s_cc[j] = row_dist2<T, D, false>(Kc + (size_t)j * D, s_c);
+    __syncthreads();
+    // rows whose D^2 may drop
+    for (int c0 = warp * kWarp; c0 < g.L; c0 += NT) {
+      const int i = c0 + lane;
+      bool need = false;
+      if (i < g.L) need = (k == 0) || !(s_cc[s_a[i]] >= 4.0 * s_d2[i] * (1.0 + 1e-9));
+      const unsigned m = __ballot_sync(kFull, need);
+      if (m) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&s_n, __popc(m));
+        base = __shfl_sync(kFull, base, 0);
+        if (need) s_list[base + __popc(m & ((1u << lane) - 1u))] = (uint16_t)i;
+      }
+    }
+    __syncthreads();
+    const int n_need = s_n;
+#pragma unroll 1
+    for (int q = tid; q < n_need; q += NT) {
+      const int i = s_list[q];
+      const double acc = row_dist2<T, D, true>(src + (size_t)i * D, s_c);
+      if (k == 0 || acc < s_d2[i]) { s_d2[i] = acc; s_a[i] = (uint16_t)k; }
+    }
+    __syncthreads();
+    if (k + 1 == g.C) break;
+    double part = 0.0;
+    for (int c0 = wr0; c0 < wr1; c0 += kWarp) part += (c0 + lane < wr1) ? s_d2[c0 + lane] : 0.0;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(kFull, part, o);
+    if (lane == 0) s_w[warp] = part;
+    if (tid == 0) s_pick = g.L - 1;
+    __syncthreads();
+    double before = 0.0, tot = 0.0;
+    for (int w = 0; w < NW; ++w) {
+      const double v = s_w[w];
+      if (w < warp) before += v;
+      tot += v;
+    }
+    int next = first;
+    if (tot > 0.0) {
+      const double thr = stream_uniform(b.seed, g.unit, g.j, 0, k + 1) * tot;
+      double run = before;
+      for (int c0 = wr0; c0 < wr1; c0 += kWarp) {
+        const int i = c0 + lane;
+        double x = i < wr1 ? s_d2[i] : 0.0;
+#pragma unroll
+        for (int o = 1; o < kWarp; o <<= 1) {
+          const double y = __shfl_up_sync(kFull, x, o);
+          if (lane >= o) x += y;
+        }
+        const unsigned hit = __ballot_sync(kFull, i < wr1 && run + x > thr);
+        if (hit) {
+          if (lane == 0) atomicMin(&s_pick, c0 + __ffs(hit) - 1);
+          break;
+        }
+        run += __shfl_sync(kFull, x, kWarp - 1);
+      }
+      __syncthreads();
+      next = s_pick;
+    }
+    __syncthreads();
+    pick = next;
+  }
+}
+
 // Slots [c_from, C) of each block start at src tokens first + (k - c_from) * T
 // (the stride initialisation, and the new slots of a warm start).
 template <typename T, int D>
@@ -735,9 +892,22 @@ __global__ void fill_tail_offsets_kernel(int32_t* off, int slots, int c_from, in
       coff[(size_t)unit * (coarse_slots + 1) + k] = (k == coarse_slots) ? slots : (k / CC_blk) * C_blk;
 }
 
-// New tail rows: perm = own id, assign = -1.
-__global__ void tail_meta_kernel(int32_t* perm, int32_t* assign, int64_t max_tokens, int64_t n0, int n_new) {
+// Appended rows of one unit (blockIdx.y): K, V rows [n0, n0 + n_new) of the
+// store from the caller's [unit][n_new] rows, perm = own id, assign = -1.  W is
+// the copy word (16 bytes when every address and row is 16-byte aligned).
+template <typename W>
+__global__ void append_kernel(const char* Kn, const char* Vn, char* Kp, char* Vp, size_t row_bytes, int64_t max_tokens,
+                              int64_t n0, int n_new, int32_t* perm, int32_t* assign) {
   const int unit = blockIdx.y;
+  const size_t words = (size_t)n_new * row_bytes / sizeof(W);
+  const W* sk = reinterpret_cast<const W*>(Kn + (size_t)unit * n_new * row_bytes);
+  const W* sv = reinterpret_cast<const W*>(Vn + (size_t)unit * n_new * row_bytes);
+  W* dk = reinterpret_cast<W*>(Kp + ((size_t)unit * max_tokens + n0) * row_bytes);
+  W* dv = reinterpret_cast<W*>(Vp + ((size_t)unit * max_tokens + n0) * row_bytes);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < words; i += (size_t)gridDim.x * blockDim.x) {
+    dk[i] = sk[i];
+    dv[i] = sv[i];
+  }
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_new; i += gridDim.x * blockDim.x) {
     perm[(size_t)unit * max_tokens + n0 + i] = (int32_t)(n0 + i);
     assign[(size_t)unit * max_tokens + n0 + i] = -1;
@@ -791,10 +961,19 @@ static cudaError_t run_lloyd(const BlockJob& b, int nbj, int units, int init_mod
   if (init != nullptr) {
     seed_given_kernel<T, D><<<dim3(64, nbj, units), 128, 0, st>>>(b, static_cast<const T*>(init));
   } else if (init_mode == MP_INIT_KMEANSPP) {
-    size_t smem = (size_t)b.L_blk * sizeof(double);
-    cudaError_t e = cudaFuncSetAttribute(kmeanspp_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kmeanspp_kernel<T, D><<<gb, kPPThreads, smem, st>>>(b);
+    const size_t smem_p = kmeanspp_pruned_smem(b.L_blk, b.C_blk);
+    if (smem_p <= 200 * 1024 && b.L_blk <= 65535 && b.C_blk <= 65535 && ((uintptr_t)b.srcK & 15u) == 0 &&
+        ((uintptr_t)b.Kc & 15u) == 0) {
+      cudaError_t e = cudaFuncSetAttribute(kmeanspp_pruned_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem_p);
+      if (e != cudaSuccess) return e;
+      kmeanspp_pruned_kernel<T, D><<<gb, kPPrThreads, smem_p, st>>>(b);
+    } else {
+      size_t smem = (size_t)b.L_blk * sizeof(double);
+      cudaError_t e = cudaFuncSetAttribute(kmeanspp_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      kmeanspp_kernel<T, D><<<gb, kPPThreads, smem, st>>>(b);
+    }
   } else {
     seed_stride_kernel<T, D><<<dim3(64, nbj, units), 128, 0, st>>>(b, L_old_tokens);
   }
@@ -966,17 +1145,21 @@ mp_status update_impl(mp_index* idx, const void* K_new, const void* V_new, int32
   if (fired) *fired = 0;
   cudaError_t e = cudaSuccess;
   if (n_new > 0) {
+    // one launch per append: rows, perm and assign of the new tail
     char* Kp = static_cast<char*>(ws_ptr(idx, S_KP));
     char* Vp = static_cast<char*>(ws_ptr(idx, S_VP));
-    e = cudaMemcpy2DAsync(Kp + (size_t)n0 * row_bytes, (size_t)c.max_tokens * row_bytes, K_new,
-                          (size_t)n_new * row_bytes, (size_t)n_new * row_bytes, units, cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(Vp + (size_t)n0 * row_bytes, (size_t)c.max_tokens * row_bytes, V_new,
-                            (size_t)n_new * row_bytes, (size_t)n_new * row_bytes, units, cudaMemcpyDeviceToDevice, st);
-    if (e != cudaSuccess) return MP_ECUDA;
-    tail_meta_kernel<<<dim3((n_new + 255) / 256, units), 256, 0, st>>>(
-        static_cast<int32_t*>(ws_ptr(idx, S_PERM)), static_cast<int32_t*>(ws_ptr(idx, S_ASSIGN)), c.max_tokens, n0,
-        n_new);
+    int32_t* perm = static_cast<int32_t*>(ws_ptr(idx, S_PERM));
+    int32_t* asg = static_cast<int32_t*>(ws_ptr(idx, S_ASSIGN));
+    const bool v16 = (((uintptr_t)K_new | (uintptr_t)V_new | (uintptr_t)Kp | (uintptr_t)Vp | row_bytes) & 15u) == 0;
+    const size_t words = (size_t)n_new * row_bytes / (v16 ? 16 : 2);
+    const int gx = (int)std::min<size_t>(std::max<size_t>((words + 255) / 256, (size_t)(n_new + 255) / 256), 1024);
+    const char* kn = static_cast<const char*>(K_new);
+    const char* vn = static_cast<const char*>(V_new);
+    if (v16)
+      append_kernel<uint4><<<dim3(gx, units), 256, 0, st>>>(kn, vn, Kp, Vp, row_bytes, c.max_tokens, n0, n_new, perm, asg);
+    else
+      append_kernel<uint16_t><<<dim3(gx, units), 256, 0, st>>>(kn, vn, Kp, Vp, row_bytes, c.max_tokens, n0, n_new, perm,
+                                                              asg);
     if (cudaGetLastError() != cudaSuccess) return MP_ECUDA;
   }
   const int64_t n1 = n0 + n_new;

@@ -116,3 +116,16 @@ def test_hierarchical_decode_matches_oracle(coarse_budget, budget, no_approx):
     oidx = H.component_index(o, K, V, lab, 5500)
     Q = synth.make_queries(1, 2, 8, 128, "bf16", seed=3)[0]
     run_decode(o, oidx, Q, budget, coarse_budget=coarse_budget, no_approx=no_approx)
+
+
+@pytest.mark.parametrize("levels", [1, 2])
+def test_4096_slot_units_decode(levels):
+    """One unit of 64K tokens at 16 tokens per centroid: 4096 slots, whose
+    selection keys fill the 48 KB default shared-memory window exactly (fp32
+    flat index on the multi-kernel path, and the hierarchical index)."""
+    dt = "f32" if levels == 1 else "bf16"
+    o = H.ocfg(B=1, Hkv=1, Hq=4, d=128, n_max=65536, T=16, L_blk=8192, levels=levels, Tc=128, dtype=dt)
+    K, V, lab = H.cache_for(o, 65536, comps=512, seed=21)
+    oidx = H.component_index(o, K, V, lab, 65536)
+    Q = synth.make_queries(1, 1, 4, 128, dt, seed=4)[0]
+    run_decode(o, oidx, Q, 512, coarse_budget=4096 if levels == 2 else 0)

@@ -220,6 +220,41 @@ def test_kmeanspp_seeding_matches_oracle_picks():
                 np.testing.assert_array_equal(ga["perm"][b, h, s:e], oidx["perm"][b, h, s:e])
 
 
+@pytest.mark.parametrize("aligned", [True, False])
+def test_kmeanspp_seeding_on_8k_blocks(aligned):
+    """512 picks over 8192 mixture keys (d 128): the seeding that skips rows
+    by the triangle inequality (16-byte aligned keys) and the full-pass seeding
+    (keys at an odd 2-byte offset) both give the oracle's picks, seen through
+    the centroids after one Lloyd iteration."""
+    o = H.ocfg(B=1, Hkv=2, Hq=8, d=128, n_max=8192, T=16, L_blk=8192, dtype="bf16", iters=1, seed=31)
+    K, V, _ = H.cache_for(o, 8192, comps=512, outliers=(4, 4.0), seed=8)
+    rec = {}
+    oidx = mp.build_index(K, V, 8192, o, record=rec)
+    g = MultipoleIndex(H.gcfg(o, init="kmeans++"))
+    Kd, Vd = H.tdev(K, "bf16"), H.tdev(V, "bf16")
+    if not aligned:
+        buf = torch.empty(Kd.numel() + 1, dtype=torch.bfloat16, device="cuda")
+        Kd = buf[1:].view(Kd.shape).copy_(Kd)
+        assert Kd.data_ptr() % 16 != 0 and Kd.is_contiguous()
+    g.build(Kd, Vd)
+    torch.cuda.synchronize()
+    assert g.check_device_error() == 0
+    ga = arrays_np(g)
+    for h in range(2):
+        X = K[0, h].astype(np.float64)
+        init = X[mp.kmeanspp_pick(X, 512, mp.stream_uniforms(31, h, 0, 0, 512))]
+        # rows within the assignment's tie band may go either way; every other
+        # row's slot, and the mean of every slot no such row touches, is exact
+        tied = rec[(0, h, 0)][0]["gap"] <= band_for(X, init)
+        assert tied.mean() < 0.01
+        ag, ao = ga["assign"][0, h, :8192], oidx["assign"][0, h, :8192]
+        np.testing.assert_array_equal(ag[~tied], ao[~tied])
+        touched = np.zeros(512, dtype=bool)
+        touched[ag[tied]] = True
+        touched[ao[tied]] = True
+        np.testing.assert_array_equal(ga["Kc"][0, h][~touched], oidx["Kc"][0, h][~touched])
+
+
 def any_tie(hist, X, init):
     return first_tie_iteration(hist, X, init) < len(hist)
 

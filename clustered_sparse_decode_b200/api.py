@@ -79,7 +79,8 @@ class MultipoleIndex:
         ib, sb = workspace_size(cfg)
         with torch.cuda.device(self.device):
             self.workspace = torch.empty(ib, dtype=torch.uint8, device=self.device)
-            self.scratch = torch.empty(sb, dtype=torch.uint8, device=self.device)
+            # zeroed once: mp_decode keeps the scratch's ticket head zero between steps
+            self.scratch = torch.zeros(sb, dtype=torch.uint8, device=self.device)
             self.h = L.MpIndex()
             c = cfg.to_c()
             L.check(self.lib.mp_index_init(ctypes.byref(c), _ptr(self.workspace), ib, ctypes.byref(self.h),
@@ -107,15 +108,14 @@ class MultipoleIndex:
 
         A flat bf16 index with at most 4096 slots per unit, fewer than 512
         units and at least 8 tokens decodes with a centroid pass and a value
-        pass (after a reset of its ticket words); the others run a longer
-        kernel pipeline.
+        pass; the others run a longer kernel pipeline.
         """
         c = self.cfg
         units = c.batch * c.kv_heads
         if (c.levels == 1 and c.dtype == "bf16" and c.head_dim in (64, 128) and self.slots <= 4096
                 and units < 512 and self.n_tokens >= 8 and c.max_tokens <= (1 << 25)
                 and units * c.max_tokens < 2 ** 31 - 1 and c.q_heads // c.kv_heads in (1, 2, 4, 8)):
-            return ["ticket reset", "centroid pass + value pass"]
+            return ["centroid pass + value pass"]
         if c.levels == 1:
             return ["centroid pass", "select", "token pass", "combine"]
         return ["coarse pass", "coarse select", "fine pass", "fine select", "token pass", "combine"]
@@ -272,9 +272,18 @@ class MultipoleIndex:
                                          _stream(stream)), "mp_index_import")
 
     def check_device_error(self, stream=None):
-        """Synchronise and return the device error word (0 = none); clears it."""
+        """Synchronise and return the device error word (0 = none); clears it.
+
+        After an error the ticket heads of this index's decode scratch and of
+        the library's own scratch are zeroed again (a step that stopped early
+        may have left arrival counters behind)."""
         code = ctypes.c_int32(0)
         st = self.lib.mp_check_device_error(ctypes.byref(self.h), ctypes.byref(code), _stream(stream))
         if st not in (L.MP_OK, L.MP_EDEVICE):
             L.check(st, "mp_check_device_error")
+        if code.value != 0:
+            with torch.cuda.device(self.device):
+                self.scratch[:L.MP_SCRATCH_TICKET_BYTES].zero_()
+                L.check(self.lib.mp_decode_static_reset(_stream(stream)), "mp_decode_static_reset")
+                torch.cuda.synchronize(self.device)
         return code.value

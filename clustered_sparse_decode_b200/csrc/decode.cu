@@ -591,7 +591,7 @@ static DecodeLayout decode_layout(const mp_config& c, int slots, int coarse_slot
   L.cap_fine = coarse_slots;
   L.cap_sub = slots;
   L.cap_csub = coarse_slots;
-  size_t cur = 0;
+  size_t cur = kScratchTicketBytes;   // the two-pass decode's ticket words stay untouched
   const size_t rows = (size_t)L.units * L.G;
   L.o_pm = cur; cur = align256(cur + rows * L.P * 4);
   L.o_pl = cur; cur = align256(cur + rows * L.P * 4);

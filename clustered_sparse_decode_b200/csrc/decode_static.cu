@@ -59,7 +59,18 @@ extern "C" mp_status mp_decode_static(const mp_index* idx, const void* Q, void* 
   void* scratch = nullptr;
   mp_status s = scratch_address(dev, &scratch);
   if (s != MP_OK) return s;
-  // Nothing in the scratch has to start at zero: every byte a decode step reads
-  // was written earlier in the same step.
+  // Apart from the ticket head (zero-initialised with the array and left zero
+  // by every finished step), every byte a decode step reads was written
+  // earlier in the same step.
   return decode_impl(idx, Q, O, p, scratch, MP_STATIC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" mp_status mp_decode_static_reset(void* stream) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MP_ECUDA;
+  void* scratch = nullptr;
+  mp_status s = scratch_address(dev, &scratch);
+  if (s != MP_OK) return s;
+  return cudaMemsetAsync(scratch, 0, kScratchTicketBytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MP_OK
+                                                                                                        : MP_ECUDA;
 }

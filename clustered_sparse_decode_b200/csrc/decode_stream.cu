@@ -837,6 +837,9 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
   const long long lo = share_lo(c, NCH, grid), hi = share_lo(c + 1, NCH, grid);
   const long long t_start = gtimer();
   auto aux = [&](int slot) { return smem + Gm::OFF_AUX + slot * Gm::AUX; };
+  // value-pass tickets start at zero (the value pass reads them after this grid completes)
+  if (c == 0)
+    for (int u = threadIdx.x; u < a.units; u += blockDim.x) a.ctl[a.units + u] = 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {
@@ -958,7 +961,9 @@ __global__ void __launch_bounds__(kCT + kWarp, 1) centroid_pass(const __grid_con
       if (threadIdx.x == 0) bc[0] = ticket(a.ctl + u);
       cbar();
       const int t = bc[0];
-      if (t == shares_of((long long)u * a.cpu, (long long)(u + 1) * a.cpu, NCH, grid) - 1)
+      const int ncs = shares_of((long long)u * a.cpu, (long long)(u + 1) * a.cpu, NCH, grid);
+      if ((t < 0 || t >= ncs) && threadIdx.x == 0) set_error(a.err, E_SCRATCH);
+      if (t == ncs - 1)
         select_unit<D, G, SG>(a, u, red, reinterpret_cast<int*>(smem + Gm::OFF_WPRE));
       cbar();
     }
@@ -1026,6 +1031,9 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
   }
   // everything below reads what the centroid pass wrote
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // the centroid pass is complete: its tickets go back to zero for the next step
+  if (c == 0)
+    for (int u = threadIdx.x; u < a.units; u += blockDim.x) a.ctl[u] = 0;
   if (warp < kCW) {
     // per-unit weights and their prefix
     long long* wtmp = reinterpret_cast<long long*>(smem);   // the first slot is not in use yet
@@ -1271,9 +1279,12 @@ __global__ void __launch_bounds__(kCT + kVP * kWarp, 1) value_pass(const __grid_
       if (threadIdx.x == 0) bc[0] = ticket(a.ctl + a.units + u);
       cbar();
       const int nvs = shares_of(wpre[u], wpre[u + 1], WT, grid);
+      if ((bc[0] < 0 || bc[0] >= nvs) && threadIdx.x == 0) set_error(a.err, E_SCRATCH);
       if (bc[0] == nvs - 1) {
-        // last share of the unit: merge all its partials (centroid and value pass) into the output rows
+        // last share of the unit: merge all its partials (centroid and value pass) into the output rows;
+        // every value share of the unit has taken its ticket, which goes back to zero
         combine_unit<D, G>(a, u, grid, wpre[u], nvs, WT);
+        if (threadIdx.x == 0) a.ctl[a.units + u] = 0;
       }
       cbar();
     }
@@ -1300,7 +1311,10 @@ static StreamLayout stream_layout(const mp_config& c, int slots) {
   L.npart = 2 * (stream::kMaxGrid + (int)U) * stream::kCW;
   L.SG = (G + 3) / 4 * 4;
   L.capc = ((slots + 3) & ~3) + 64;
-  size_t cur = 0;
+  static_assert(2 * stream::kMaxUnits * 4 <= kScratchTicketBytes, "ticket words");
+  L.o_ctl = 0;                                        // ticket words: zero between steps
+  L.ctl_bytes = kScratchTicketBytes;
+  size_t cur = kScratchTicketBytes;
   L.o_S = cur; cur = a256(cur + U * slots * L.SG * 4);
   L.o_shat = cur; cur = a256(cur + U * slots * 4);
   L.o_tok = cur; cur = a256(cur + U * (size_t)c.max_tokens * 4);
@@ -1310,9 +1324,6 @@ static StreamLayout stream_layout(const mp_config& c, int slots) {
   L.o_pm = cur; cur = a256(cur + (size_t)L.npart * G * 4);
   L.o_pl = cur; cur = a256(cur + (size_t)L.npart * G * 4);
   L.o_pacc = cur; cur = a256(cur + (size_t)L.npart * G * D * 4);
-  L.o_ctl = cur;                                      // ticket words, reset before every step
-  L.ctl_bytes = 2 * U * 4;
-  cur = a256(cur + L.ctl_bytes);
   L.bytes = cur;
   return L;
 }
@@ -1421,7 +1432,11 @@ static cudaError_t launch_stream_d(int G, const stream::Args& a, int grid, cudaS
   return cudaErrorInvalidValue;
 }
 
-// The flat bf16 decode step: a memset of the ticket words and two kernels.
+// The flat bf16 decode step: two kernels.  The centroid tickets at the head of
+// the scratch are zero on entry; the value pass zeroes them again (after the
+// centroid pass has completed), the centroid pass zeroes the value tickets at
+// its start and each unit's combining CTA its own after the combine, so a
+// finished step leaves the whole ticket head zero.
 mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
                         size_t scratch_bytes, float scale, cudaStream_t st) {
   const mp_config& c = idx->cfg;
@@ -1481,11 +1496,15 @@ mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_de
       cudaEventRecord(static_cast<cudaEvent_t>(prm->phase_events[i]), st);
   };
   phase(0);
-  if (cudaMemsetAsync(base + L.o_ctl, 0, L.ctl_bytes, st) != cudaSuccess) return MP_ECUDA;
-  phase(1);
   cudaError_t e = D == 128 ? launch_stream_d<128>(G, a, grid, st) : launch_stream_d<64>(G, a, grid, st);
-  phase(2);
-  return e == cudaSuccess ? MP_OK : MP_ECUDA;
+  phase(1);
+  if (e != cudaSuccess) {
+    // a launch that did not happen may leave the centroid tickets taken
+    cudaGetLastError();
+    cudaMemsetAsync(base + L.o_ctl, 0, L.ctl_bytes, st);
+    return MP_ECUDA;
+  }
+  return MP_OK;
 }
 
 }  // namespace mp

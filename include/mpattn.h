@@ -28,7 +28,10 @@
  *    exceeded) and leave the index unchanged.  A launch failure returns
  *    MP_ECUDA.  Kernels never trap: a data-dependent fault found on the device
  *    (e.g. corrupt offsets in an imported index) sets a device error word and
- *    skips the faulty access; mp_check_device_error reports it.
+ *    skips the faulty access; mp_check_device_error reports it.  Its bits:
+ *    1 a run offset or slot outside the index, 2 an inconsistent internal run
+ *    list, 4 a bounded wait gave up, 8 a per-unit kernel limit exceeded,
+ *    16 a decode scratch whose ticket head was not zero.
  *  - An index is not thread-safe: one host thread, one stream at a time.
  */
 #ifndef MPATTN_H
@@ -206,6 +209,17 @@ mp_status mp_cluster_assign(const mp_index* idx, const void* K, int32_t n, int32
 mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
                     void* d_scratch, size_t scratch_bytes, void* stream);
 
+/* The first MP_SCRATCH_TICKET_BYTES of every decode scratch hold the arrival
+ * counters of the two-pass decode kernels (an implementation detail, no
+ * counterpart in the paper).  They must be zero before the first mp_decode
+ * that uses the buffer (e.g. one cudaMemset when it is allocated); every
+ * finished decode leaves them zero, so a scratch can serve any number of
+ * steps and indices without a reset.  After mp_check_device_error has
+ * reported an error, zero them again (mp_decode_static_reset for the
+ * library's own scratch).  A decode that finds them non-zero sets bit 16 of
+ * the device error word. */
+#define MP_SCRATCH_TICKET_BYTES 4096u
+
 /* Size of the library's own decode scratch used by mp_decode_static. */
 #define MP_STATIC_SCRATCH_BYTES (32u << 20)
 
@@ -223,11 +237,16 @@ mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
  *  - All calls on a device share the one array and it keeps the last call's
- *    contents (nothing in it needs to start at zero).  Calls that overlap on
- *    the GPU (other streams, other threads, other indices) race on it: order
- *    them, e.g. on one stream. */
+ *    contents; its ticket head (MP_SCRATCH_TICKET_BYTES) starts zeroed.
+ *    Calls that overlap on the GPU (other streams, other threads, other
+ *    indices) race on it: order them, e.g. on one stream. */
 mp_status mp_decode_static(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
                            void* stream);
+
+/* Zero the ticket head of the library's own decode scratch on the current
+ * device (enqueued on `stream`), e.g. after mp_check_device_error reported an
+ * error for a mp_decode_static call. */
+mp_status mp_decode_static_reset(void* stream);
 
 /* Device pointers of the index arrays (layouts above). */
 mp_status mp_index_export(const mp_index* idx, mp_index_view* view);

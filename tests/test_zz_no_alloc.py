@@ -49,3 +49,25 @@ def test_static_scratch_rejects_configurations_that_do_not_fit():
     # the regular entry point still works for it
     idx.decode(Q, 16)
     torch.cuda.synchronize()
+
+
+def test_one_scratch_serves_indices_of_different_shapes():
+    """The library's array serves, in turn, two-pass indices of 4 and 16 units
+    and a multi-kernel (fp32) index, many steps each: the ticket head stays
+    zero between steps (no error bit, results equal to mp_decode's)."""
+    shapes = [("bf16", 2, 2), ("bf16", 4, 4), ("f32", 2, 2)]
+    runs = []
+    for s, (dtype, B, Hkv) in enumerate(shapes):
+        o = H.ocfg(B=B, Hkv=Hkv, Hq=4 * Hkv, d=128, n_max=4096, T=16, L_blk=2048, iters=2, dtype=dtype, seed=s)
+        K, V, _ = H.cache_for(o, 3000 + 100 * s, comps=48, seed=s)
+        idx = MultipoleIndex(H.gcfg(o))
+        idx.build(H.tdev(K[:, :, :3000 + 100 * s], dtype), H.tdev(V[:, :, :3000 + 100 * s], dtype))
+        Q = H.tdev(synth.make_queries(1, B, 4 * Hkv, 128, dtype, seed=s)[0], dtype)
+        runs.append((idx, Q, idx.decode(Q, 200).clone()))
+    for rep in range(5):
+        for idx, Q, ref in runs[::-1] if rep % 2 else runs:
+            got = idx.decode_static(Q, 200)
+            torch.cuda.synchronize()
+            assert torch.equal(got, ref)
+    for idx, _, _ in runs:
+        assert idx.check_device_error() == 0

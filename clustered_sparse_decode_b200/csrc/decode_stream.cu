@@ -698,14 +698,105 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
   const int mode = (a.budget <= 0 || W == 0) ? 0 : (W <= a.budget ? 1 : 2);
   uint32_t tau = 0u;
   int need = 0, ntie = 0;
+  bool resolved = false;
+  int above = 0;                                            // weight of the keys above tau
   if (mode == 2) {
+    // First try: 256 bins of equal width in score between the smallest and the
+    // largest candidate score (the bin index is monotone in the score, so a
+    // higher bin holds only higher keys); one warp finds the bin where the
+    // weight from the top crosses the budget, and if at most 32 candidates fall
+    // in it, sorts them by (key descending, slot ascending) and takes tau from
+    // the running weight.  Otherwise the radix descent below decides.
+    const float smin = key_score(kmin), smax = key_score(kmax);
+    const float span = smax - smin, inv = 256.f / span;
+    if (isfinite(smin) && isfinite(smax) && span > 0.f && isfinite(span) && isfinite(inv)) {
+      auto fbin = [&](uint32_t kk) { return min(255, (int)((key_score(kk) - smin) * inv)); };
+      int* lst = hist + 256;                                // [32][3] candidates of the crossing bin
+      for (int i = tid; i < 256; i += kCT) hist[i] = 0;
+      if (tid == 0) red[3] = 0;
+      cbar();
+#pragma unroll
+      for (int k = 0; k < kMaxSpt; ++k)
+        if (w[k] > 0) atomicAdd(hist + fbin(key[k]), w[k]);
+      cbar();
+      if (warp == 0) {
+        int bl[8], ls = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { bl[i] = hist[8 * lane + i]; ls += bl[i]; }
+        int suf = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(kFull, suf, o);
+          if (lane + o < 32) suf += y;
+        }
+        int run = suf - ls, found = -1, ab = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (found < 0 && run + bl[i] >= a.budget) { found = 8 * lane + i; ab = run; }
+          run += bl[i];
+        }
+        const unsigned m = __ballot_sync(kFull, found >= 0);
+        const int src = 31 - __clz(m);
+        const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
+        if (lane == 0) { red[0] = fb; red[1] = fa; }
+      }
+      cbar();
+      const int fb = red[0], ab = red[1];
+#pragma unroll
+      for (int k = 0; k < kMaxSpt; ++k)
+        if (w[k] > 0 && fbin(key[k]) == fb) {
+          const int pos = atomicAdd(red + 3, 1);
+          if (pos < 32) { lst[3 * pos] = (int)key[k]; lst[3 * pos + 1] = s0 + k; lst[3 * pos + 2] = w[k]; }
+        }
+      cbar();
+      const int nc = red[3];
+      if (nc <= 32) {
+        if (warp == 0) {
+          // lane l holds candidate l; empty lanes sort last with weight 0
+          uint64_t v = lane < nc ? ((uint64_t)(uint32_t)lst[3 * lane] << 32) | (uint32_t)(0xffffffffu - (uint32_t)lst[3 * lane + 1])
+                                 : 0ull;
+          int wl = lane < nc ? lst[3 * lane + 2] : 0;
+          // bitonic sort, descending
+#pragma unroll
+          for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+              const uint64_t ov = __shfl_xor_sync(kFull, v, jj);
+              const int ow = __shfl_xor_sync(kFull, wl, jj);
+              const bool up = ((lane & kk) == 0) == ((lane & jj) == 0);   // this lane keeps the larger
+              if (up ? ov > v : ov < v) { v = ov; wl = ow; }
+            }
+          }
+          int inc = wl;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += y;
+          }
+          const unsigned cross = __ballot_sync(kFull, lane < nc && ab + inc >= a.budget);
+          const uint32_t t = (uint32_t)(__shfl_sync(kFull, v, __ffs(cross) - 1) >> 32);
+          const uint32_t kl = (uint32_t)(v >> 32);
+          const int gt = __reduce_add_sync(kFull, lane < nc && kl > t ? wl : 0);
+          const int nt = __popc(__ballot_sync(kFull, lane < nc && kl == t));
+          if (lane == 0) { red[0] = (int)t; red[1] = ab + gt; red[2] = nt; }
+        }
+        cbar();
+        tau = (uint32_t)red[0];
+        above = red[1];
+        ntie = red[2];
+        resolved = true;
+      }
+      cbar();
+    }
+  }
+  if (mode == 2 && !resolved) {
     // Radix descent over the interval [lo, lo + 2^nb) holding all candidates,
     // 8 bits a level: a 256-bin histogram of weights (and, on the last level,
     // where bins are single key values, of key counts), then warp 0 finds the
     // bin where the weight from the top crosses the budget.
     uint32_t lo = kmin;
     int nb = kmax == kmin ? 0 : 32 - __clz(kmax - kmin);
-    int above = 0;                                          // weight of the keys above the interval
+    above = 0;                                              // weight of the keys above the interval
     int* hcnt = hist + 256;
     ntie = -1;                                              // keys at tau: unknown unless a level ends on single keys
     while (nb > 0) {
@@ -753,8 +844,8 @@ __device__ void select_unit(const Args& a, int u, int* red, int* hist) {
       cbar();
     }
     tau = lo;
-    need = a.budget - above;   // >= 1 tokens still to take among the ties at tau
   }
+  if (mode == 2) need = a.budget - above;   // >= 1 tokens still to take among the ties at tau
   int tw = 0;
   if (mode == 2) {
 #pragma unroll

@@ -95,6 +95,10 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// the score of an ordered key (inverse of ordered_key)
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 __device__ __forceinline__ void set_error(int32_t* err, int32_t bit) {
   if (err) atomicOr(err, bit);

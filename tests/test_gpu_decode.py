@@ -129,3 +129,45 @@ def test_4096_slot_units_decode(levels):
     oidx = H.component_index(o, K, V, lab, 65536)
     Q = synth.make_queries(1, 1, 4, 128, dt, seed=4)[0]
     run_decode(o, oidx, Q, 512, coarse_budget=4096 if levels == 2 else 0)
+
+
+def brute_selection(score, count, budget):
+    """Clusters by score descending (ties: lower slot), shortest prefix whose
+    token count reaches the budget; every non-empty cluster if it never does."""
+    order = sorted(np.nonzero(count > 0)[0].tolist(), key=lambda c: (-score[c], c))
+    sel, tot = set(), 0
+    for c in order:
+        if budget <= 0 or tot >= budget:
+            break
+        sel.add(c)
+        tot += int(count[c])
+    return sel
+
+
+@pytest.mark.parametrize("budget", [1, 100, 1124, 3000, 4096, 5000])
+def test_selection_with_exact_score_ties(budget):
+    """The selection as a function of the scores it reports: groups of 64 and of
+    4 clusters with identical keys (exact score ties at the crossing, more and
+    fewer candidates than one warp resolves) and one unit of distinct keys."""
+    o = H.ocfg(B=1, Hkv=3, Hq=12, d=128, n_max=4096, T=16, L_blk=4096)
+    rng = np.random.default_rng(12)
+    K = np.empty((1, 3, 4096, 128), dtype=np.float32)
+    for h, grp in enumerate((64, 4, 1)):
+        base = synth._cast(rng.standard_normal((256 // grp, 128)), "bf16")
+        K[0, h] = np.repeat(base, 16 * grp, axis=0)
+    V = synth._cast(rng.standard_normal((1, 3, 4096, 128)), "bf16")
+    a = np.broadcast_to(np.arange(4096) // 16, (1, 3, 4096))
+    oidx = mp.index_from_assignment(K, V, 4096, o, a)
+    gidx = MultipoleIndex(H.gcfg(o))
+    H.upload_index(gidx, oidx)
+    mask = torch.zeros((1, 3, gidx.slots), dtype=torch.uint8, device="cuda")
+    scores = torch.empty((1, 3, gidx.slots), dtype=torch.float32, device="cuda")
+    Q = synth.make_queries(1, 1, 12, 128, "bf16", seed=6)[0]
+    gidx.decode(H.tdev(Q, "bf16"), budget, sel_mask=mask, scores=scores)
+    torch.cuda.synchronize()
+    assert gidx.check_device_error() == 0
+    count = np.diff(oidx["off"][0], axis=-1)
+    for h in range(3):
+        want = brute_selection(scores[0, h].cpu().numpy(), count[h], budget)
+        got = set(np.nonzero(mask[0, h].cpu().numpy())[0].tolist())
+        assert got == want, f"unit {h}"

@@ -310,18 +310,17 @@ def run_ours(args, w):
     gbs = tot_bytes / tot_time / 1e9
     ms_per_step = 1e3 * tot_time / args.steps
 
-    # end to end through the C ABI: Q from pinned host memory, O back to the host, every step
+    # end to end through the C ABI with host buffers: each step's Q is read from
+    # pinned host memory (by the library's staging kernel) and O is written back
+    # to pinned host memory (by the decode's combine), and the host waits for it
     Qpin = torch.from_numpy(Qh).to(tdt).pin_memory() if w["dtype"] == "bf16" else torch.from_numpy(Qh).pin_memory()
     Opin = torch.empty((B, Hq, d), dtype=tdt).pin_memory()
-    Qdev = torch.empty((B, Hq, d), dtype=tdt, device=dev)
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         flush_l2()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        Qdev.copy_(Qpin[i], non_blocking=True)
-        idx.decode(Qdev, budget, coarse_budget=cb, out=O)
-        Opin.copy_(O, non_blocking=True)
+        idx.decode(Qpin[i], budget, coarse_budget=cb, out=Opin)
         b_.record(stream)
         b_.synchronize()
         if i >= args.warmup:

@@ -174,6 +174,10 @@ class MultipoleIndex:
                stream=None):
         """One decode step: O [B, Hq, d] for Q [B, Hq, d] (mp_decode).
 
+        Q and out may be device tensors or page-locked (pinned) host tensors;
+        a host Q is copied in by the library's kernel and a host out is written
+        over the host link, within the call's stream work.
+
         Optional device outputs: sel_mask / coarse_sel_mask (uint8 [B, Hkv, slots]),
         scores / coarse_scores (float32 [B, Hkv, slots]).  phase_events: torch.cuda.Event
         objects (already recorded once) that the library records at its kernel boundaries.
@@ -182,8 +186,14 @@ class MultipoleIndex:
         want = (c.batch, c.q_heads, c.head_dim)
         if tuple(Q.shape) != want or Q.dtype != c.torch_dtype or not Q.is_contiguous():
             raise ValueError(f"Q must be a contiguous {c.torch_dtype} tensor of shape {want}")
+        if Q.device.type == "cpu" and not Q.is_pinned():
+            raise ValueError("a host Q must be in page-locked memory (pin_memory())")
         if out is None:
-            out = torch.empty_like(Q)
+            out = torch.empty_like(Q, pin_memory=Q.device.type == "cpu")
+        elif (tuple(out.shape) != want or out.dtype != c.torch_dtype or not out.is_contiguous()
+              or (out.device.type == "cpu" and not out.is_pinned())):
+            raise ValueError(f"out must be a contiguous {c.torch_dtype} tensor of shape {want}, "
+                             "on the device or in page-locked host memory")
         p = L.MpDecodeParams()
         p.budget = int(budget)
         p.coarse_budget = int(coarse_budget)

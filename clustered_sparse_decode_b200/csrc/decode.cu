@@ -613,9 +613,38 @@ bool stream_supported(const mp_config& c, int slots, int64_t n_tokens);
 mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
                         size_t scratch_bytes, float scale, cudaStream_t st);
 
-// Both decode paths place their scratch from the start of the buffer; one call uses one of them.
+// Both decode paths place their scratch from the start of the buffer (one call
+// uses one of them); after them, room for a device copy of Q when the caller's
+// Q is page-locked host memory.
+static size_t q_stage_offset(const mp_config& c, int slots, int coarse_slots) {
+  return align256(std::max(decode_layout(c, slots, coarse_slots).bytes, stream_scratch_bytes(c, slots)));
+}
+static size_t q_bytes(const mp_config& c) {
+  return (size_t)c.batch * c.q_heads * c.head_dim * elem_bytes(c.dtype);
+}
 size_t decode_scratch_bytes(const mp_config& c, int slots, int coarse_slots) {
-  return std::max(decode_layout(c, slots, coarse_slots).bytes, stream_scratch_bytes(c, slots));
+  return q_stage_offset(c, slots, coarse_slots) + align256(q_bytes(c));
+}
+
+// Q from page-locked host memory into the device: plain loads over the host link.
+template <typename W>
+__global__ void stage_q_kernel(const W* __restrict__ src, W* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
+// Where Q and O live: device (or managed) memory, or page-locked host memory
+// that the device reaches through the unified address space.  Anything else
+// (pageable host memory, unknown pointers) is refused.
+static mp_status locate(const void* p, bool* host) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return MP_EINVAL;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) { *host = false; return MP_OK; }
+  if (at.type == cudaMemoryTypeHost && at.devicePointer == p) { *host = true; return MP_OK; }
+  return MP_EINVAL;
 }
 
 static RunList runlist_at(char* base, const size_t o[3], int cap) {
@@ -688,8 +717,36 @@ static void record_phase(const mp_decode_params* prm, int i, cudaStream_t st) {
     cudaEventRecord(static_cast<cudaEvent_t>(prm->phase_events[i]), st);
 }
 
+static mp_status decode_paths(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
+                              void* scratch, size_t scratch_bytes, cudaStream_t st);
+
 mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
                       void* scratch, size_t scratch_bytes, cudaStream_t st) {
+  const mp_config& c = idx->cfg;
+  bool q_host = false, o_host = false;
+  if (locate(Q, &q_host) != MP_OK || locate(O, &o_host) != MP_OK) return MP_EINVAL;
+  (void)o_host;   // the output is written in place either way (stores over the host link for host memory)
+  if (q_host) {
+    const size_t off = q_stage_offset(c, idx->slots, idx->coarse_slots), nb = q_bytes(c);
+    if (scratch_bytes < off + nb) return MP_ENOSPC;
+    void* qd = static_cast<char*>(scratch) + off;
+    if (((uintptr_t)Q & 15u) == 0) {
+      const size_t n = nb / 16;
+      stage_q_kernel<uint4><<<(unsigned)std::min<size_t>((n + 255) / 256, 256), 256, 0, st>>>(
+          static_cast<const uint4*>(Q), static_cast<uint4*>(qd), n);
+    } else {
+      const size_t n = nb / 2;
+      stage_q_kernel<uint16_t><<<(unsigned)std::min<size_t>((n + 255) / 256, 256), 256, 0, st>>>(
+          static_cast<const uint16_t*>(Q), static_cast<uint16_t*>(qd), n);
+    }
+    if (cudaGetLastError() != cudaSuccess) return MP_ECUDA;
+    Q = qd;
+  }
+  return decode_paths(idx, Q, O, prm, scratch, scratch_bytes, st);
+}
+
+static mp_status decode_paths(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
+                              void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const mp_config& c = idx->cfg;
   // flat bf16 index: the one-kernel streaming path (decode_stream.cu)
   if (stream_supported(c, idx->slots, idx->n_tokens)) {

@@ -205,7 +205,14 @@ mp_status mp_cluster_assign(const mp_index* idx, const void* K, int32_t n, int32
  * the coarse clusters are selected first (coarse_budget), fine clusters are
  * scored and selected only inside selected coarse clusters, and unselected
  * coarse clusters contribute coarse centroid terms.  Accumulation is fp32;
- * O is written in dtype.  `d_scratch` must hold decode_scratch_bytes. */
+ * O is written in dtype.  `d_scratch` must hold decode_scratch_bytes.
+ * Q and O are device memory, or page-locked host memory mapped into the
+ * unified address space (cudaHostAlloc, cudaMallocHost; the benchmark's
+ * host-buffer path): a host Q is copied into the scratch by a library kernel,
+ * a host O is written in place over the host link, both within the stream
+ * work of the call.  Any other pointer (pageable host memory) returns
+ * MP_EINVAL before anything is launched.  The optional outputs in `params`
+ * are device memory. */
 mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
                     void* d_scratch, size_t scratch_bytes, void* stream);
 

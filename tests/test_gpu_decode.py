@@ -5,12 +5,15 @@ decode parity is checked independently of clustering parity.  Outputs are
 compared element by element (max-abs 2e-2 for bf16 inputs, 1e-4 for fp32);
 selected sets must match exactly unless a score tie within 1e-5 decides them.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
 
 import helpers as H
 from clustered_sparse_decode_b200 import MultipoleIndex, synth
+from clustered_sparse_decode_b200 import _lib as L
 from oracle import multipole as mp
 
 pytestmark = pytest.mark.gpu
@@ -171,3 +174,38 @@ def test_selection_with_exact_score_ties(budget):
         want = brute_selection(scores[0, h].cpu().numpy(), count[h], budget)
         got = set(np.nonzero(mask[0, h].cpu().numpy())[0].tolist())
         assert got == want, f"unit {h}"
+
+
+@pytest.mark.parametrize("dtype,levels", [("bf16", 1), ("f32", 1), ("bf16", 2)])
+def test_host_buffers_give_the_device_result(dtype, levels):
+    """Q and O in pinned host memory (Q staged by the library's kernel, O written
+    over the host link) give the bits of the device-buffer call; pageable host
+    memory is refused before anything is launched."""
+    o = H.ocfg(B=2, Hkv=2, Hq=8, d=128, n_max=4096, T=16, L_blk=2048, levels=levels, Tc=128, dtype=dtype, seed=2)
+    K, V, lab = H.cache_for(o, 4000, comps=64, seed=4)
+    oidx = H.component_index(o, K, V, lab, 4000)
+    gidx = MultipoleIndex(H.gcfg(o))
+    H.upload_index(gidx, oidx)
+    Q = H.tdev(synth.make_queries(1, 2, 8, 128, dtype, seed=9)[0], dtype)
+    ref = gidx.decode(Q, 300, coarse_budget=1200)
+    Qh = Q.cpu().pin_memory()
+    Oh = gidx.decode(Qh, 300, coarse_budget=1200)
+    torch.cuda.synchronize()
+    assert Oh.device.type == "cpu" and Oh.is_pinned()
+    assert torch.equal(Oh, ref.cpu())
+    # mixed: host Q into a device O, device Q into a host O
+    Od = torch.empty_like(Q)
+    gidx.decode(Qh, 300, coarse_budget=1200, out=Od)
+    Oh2 = torch.empty_like(Qh).pin_memory()
+    gidx.decode(Q, 300, coarse_budget=1200, out=Oh2)
+    torch.cuda.synchronize()
+    assert torch.equal(Od, ref) and torch.equal(Oh2, ref.cpu())
+    assert gidx.check_device_error() == 0
+    # pageable host memory: refused by the library itself
+    Qp = Q.cpu()
+    p = L.MpDecodeParams()
+    p.budget = 300
+    st = gidx.lib.mp_decode(ctypes.byref(gidx.h), ctypes.c_void_p(Qp.data_ptr()), ctypes.c_void_p(Od.data_ptr()),
+                            ctypes.byref(p), ctypes.c_void_p(gidx.scratch.data_ptr()), gidx.scratch.numel(),
+                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == L.MP_EINVAL

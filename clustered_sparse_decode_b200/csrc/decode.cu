@@ -529,25 +529,64 @@ select_kernel(SelectArgs a) {
 // Combine
 // ----------------------------------------------------------------------------
 // P: partial stride of the layout; n_used: partials written by this call.
+constexpr int kCombThreads = 512;
+constexpr int kCombMaxParts = 128;   // >= the largest P: 32 centroid + 32 fine + 64 token splits
+
+// One CTA per output row.  The partials' maxima and normalisers are read once
+// into shared memory (one thread per partial); every partial's weight
+// exp2(m_p - M) is computed there; then kCombThreads / D thread groups each
+// sum a strided share of the partials' accumulators for every column, with
+// independent loads, and the groups' sums are added in shared memory.
 template <typename T, int D>
-__global__ void combine_kernel(const float* part_m, const float* part_l, const float* part_acc, int P,
+__global__ void __launch_bounds__(kCombThreads)
+combine_kernel(const float* part_m, const float* part_l, const float* part_acc, int P,
                                int n_used, T* O) {
+  constexpr int NG = kCombThreads / D;      // partial groups
+  __shared__ float s_f[kCombMaxParts];
+  __shared__ float s_red[kCombThreads / kWarp];
+  __shared__ float s_acc[NG][D];
   const int row = blockIdx.x;   // unit * G + g == b * Hq + hq
-  const int dim = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid % kWarp, warp = tid / kWarp;
   const float* pm = part_m + (size_t)row * P;
   const float* pl = part_l + (size_t)row * P;
+  const int n = min(n_used, kCombMaxParts);
+  // 1. M = max over partials
+  const float mp = tid < n ? pm[tid] : -INFINITY;
+  float x = mp;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+  if (lane == 0) s_red[warp] = x;
+  __syncthreads();
   float M = -INFINITY;
-  for (int p = 0; p < n_used; ++p) M = fmaxf(M, pm[p]);
-  float Ls = 0.f, A = 0.f;
-  if (M != -INFINITY) {
-    for (int p = 0; p < n_used; ++p) {
-      float f = pm[p] == -INFINITY ? 0.f : exp2f(pm[p] - M);
-      Ls = fmaf(pl[p], f, Ls);
-      A = fmaf(part_acc[((size_t)row * P + p) * D + dim], f, A);
-    }
+#pragma unroll
+  for (int w = 0; w < kCombThreads / kWarp; ++w) M = fmaxf(M, s_red[w]);
+  __syncthreads();
+  // 2. weights and the normaliser
+  const float f = (tid < n && mp != -INFINITY) ? exp2f(mp - M) : 0.f;
+  if (tid < n) s_f[tid] = f;
+  float l = tid < n ? f * pl[tid] : 0.f;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(kFull, l, o);
+  if (lane == 0) s_red[warp] = l;
+  __syncthreads();
+  float Ls = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombThreads / kWarp; ++w) Ls += s_red[w];
+  // 3. accumulators: group g sums partials g, g + NG, ...
+  const int g = tid / D, dim = tid % D;
+  const float* pa = part_acc + (size_t)row * P * D + dim;
+  float A = 0.f;
+#pragma unroll 4
+  for (int p = g; p < n; p += NG) A = fmaf(pa[(size_t)p * D], s_f[p], A);
+  s_acc[g][dim] = A;
+  __syncthreads();
+  if (tid < D) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < NG; ++q) t += s_acc[q][tid];
+    const float o = (M != -INFINITY && Ls > 0.f) ? t / Ls : 0.f;
+    O[(size_t)row * D + tid] = from_f32<T>(o);
   }
-  float o = Ls > 0.f ? A / Ls : 0.f;
-  O[(size_t)row * D + dim] = from_f32<T>(o);
 }
 
 __global__ void fill_f32(float* p, size_t n, float v) {
@@ -587,6 +626,7 @@ static DecodeLayout decode_layout(const mp_config& c, int slots, int coarse_slot
   L.nsplit_f = c.levels == 2 ? 32 : 0;
   L.nsplit_t_max = kMaxSplit;
   L.P = L.nsplit_c + L.nsplit_f + L.nsplit_t_max;
+  static_assert(32 + 32 + kMaxSplit <= kCombMaxParts, "combine holds every partial's weight");
   L.cap_tok = slots + 1;
   L.cap_fine = coarse_slots;
   L.cap_sub = slots;
@@ -702,12 +742,13 @@ static cudaError_t launch_select(const SelectArgs& a, int units, cudaStream_t st
 
 static cudaError_t launch_combine(int dtype, int D, const float* pm, const float* pl, const float* pa, int P,
                                   int n_used, void* O, int rows, cudaStream_t st) {
+  if (n_used > kCombMaxParts) return cudaErrorInvalidValue;
   if (dtype == MP_BF16) {
-    if (D == 128) combine_kernel<__nv_bfloat16, 128><<<rows, 128, 0, st>>>(pm, pl, pa, P, n_used, (__nv_bfloat16*)O);
-    else combine_kernel<__nv_bfloat16, 64><<<rows, 64, 0, st>>>(pm, pl, pa, P, n_used, (__nv_bfloat16*)O);
+    if (D == 128) combine_kernel<__nv_bfloat16, 128><<<rows, kCombThreads, 0, st>>>(pm, pl, pa, P, n_used, (__nv_bfloat16*)O);
+    else combine_kernel<__nv_bfloat16, 64><<<rows, kCombThreads, 0, st>>>(pm, pl, pa, P, n_used, (__nv_bfloat16*)O);
   } else {
-    if (D == 128) combine_kernel<float, 128><<<rows, 128, 0, st>>>(pm, pl, pa, P, n_used, (float*)O);
-    else combine_kernel<float, 64><<<rows, 64, 0, st>>>(pm, pl, pa, P, n_used, (float*)O);
+    if (D == 128) combine_kernel<float, 128><<<rows, kCombThreads, 0, st>>>(pm, pl, pa, P, n_used, (float*)O);
+    else combine_kernel<float, 64><<<rows, kCombThreads, 0, st>>>(pm, pl, pa, P, n_used, (float*)O);
   }
   return cudaGetLastError();
 }

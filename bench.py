@@ -533,7 +533,7 @@ def traffic_for(kernel, workload):
         parts = [x.strip() for x in line.strip().strip("|").split("|")]
         if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload:
             try:
-                if parts[3] != source_digest():
+                if parts[3] != source_digest(kernel):
                     return None
                 return float(parts[2])
             except ValueError:
@@ -541,11 +541,18 @@ def traffic_for(kernel, workload):
     return None
 
 
-def source_digest():
+# the sources of each kernel whose traffic profiles/traffic.md records
+KERNEL_SOURCES = {"centroid pass + value pass": ("decode_stream.cu", "mp_internal.cuh")}
+
+
+def source_digest(kernel=None):
+    """sha256 prefix of the kernel's source files (all of csrc/ for an unlisted kernel)."""
     import hashlib
+    csrc = os.path.join(ROOT, "clustered_sparse_decode_b200", "csrc")
+    files = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc))
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "clustered_sparse_decode_b200", "csrc"))):
-        h.update(open(os.path.join(ROOT, "clustered_sparse_decode_b200", "csrc", f), "rb").read())
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 
 

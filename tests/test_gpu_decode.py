@@ -209,3 +209,73 @@ def test_host_buffers_give_the_device_result(dtype, levels):
                             ctypes.byref(p), ctypes.c_void_p(gidx.scratch.data_ptr()), gidx.scratch.numel(),
                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == L.MP_EINVAL
+
+
+def test_full_size_bench_launch_sampled_units():
+    """The default bench workload at full size (batch 16, 8 KV / 32 query
+    heads, 32768 tokens, 2048 slots per head, budget 1638, bf16) in the bench's
+    launch configuration (one CTA per SM over all 128 units).  The index holds
+    8 distinct oracle-built heads (mixture components as clusters), tiled over
+    the 128 units; every unit gets its own queries; 8 units spread over the
+    grid's shares are checked against the oracle (selection and outputs)."""
+    w = synth.workload("batch16_32k_sparse95")
+    B, Hkv, Hq, d, n = w["B"], w["Hkv"], w["Hq"], w["d"], w["n"]
+    G = Hq // Hkv
+    o1 = H.ocfg(B=1, Hkv=1, Hq=G, d=d, n_max=n, T=w["T"], L_blk=w["L_blk"])
+    heads = []
+    for s in range(8):
+        K, V, lab = synth.make_cache(1, 1, n, d, w["comps"], w["sigma"], radius=w["radius"], outliers=w["outliers"],
+                                     dtype="bf16", seed=w["seed"] + 17 * s)
+        heads.append(H.component_index(o1, K, V, lab, n))
+    src = torch.arange(B * Hkv) % 8
+    arr = {}
+    for k in ("Kc", "Vc", "Kp", "Vp"):
+        t = torch.stack([torch.from_numpy(np.asarray(h[k][0, 0], dtype=np.float32)) for h in heads])
+        arr[k] = t[src].reshape(B, Hkv, *t.shape[1:]).to(torch.bfloat16).cuda()
+    for k in ("off", "perm", "assign"):
+        t = torch.stack([torch.from_numpy(h[k][0, 0].astype(np.int32)) for h in heads])
+        arr[k] = t[src].reshape(B, Hkv, *t.shape[1:]).cuda()
+    cfg = H.gcfg(H.ocfg(B=B, Hkv=Hkv, Hq=Hq, d=d, n_max=n, T=w["T"], L_blk=w["L_blk"]))
+    gidx = MultipoleIndex(cfg)
+    gidx.load_arrays(arr, n, n)
+    assert gidx.decode_phases() == ["centroid pass + value pass"]
+    Q = synth.make_queries(1, B, Hq, d, "bf16", seed=71)[0]
+    mask = torch.zeros((B, Hkv, gidx.slots), dtype=torch.uint8, device="cuda")
+    scores = torch.empty((B, Hkv, gidx.slots), dtype=torch.float32, device="cuda")
+    O = H.to_np(gidx.decode(H.tdev(Q, "bf16"), w["budget"], sel_mask=mask, scores=scores))
+    torch.cuda.synchronize()
+    assert gidx.check_device_error() == 0
+    mask, scores = mask.cpu().numpy(), scores.cpu().numpy()
+    skipped = 0
+    for u in (0, 17, 38, 55, 73, 90, 111, 127):
+        b, h = divmod(u, Hkv)
+        info = {}
+        O_ref = mp.decode(heads[u % 8], Q[b:b + 1, h * G:(h + 1) * G], w["budget"], info=info)
+        skipped += H.compare_decode(o1, O[b:b + 1, h * G:(h + 1) * G], O_ref, info, mask[b:b + 1, h:h + 1],
+                                    scores[b:b + 1, h:h + 1])
+    assert skipped <= 2
+
+
+@pytest.mark.parametrize("n", [0, 5, 8, 500])
+def test_unclustered_indices(n):
+    """Indices holding only a tail (appended tokens below the update interval):
+    empty (O = 0), fewer than 8 tokens (the multi-kernel path), exactly 8 and
+    500 tokens (the two-pass path with no clusters).  Every token is attended
+    exactly: the oracle's decode of its own appended index."""
+    o = H.ocfg(B=2, Hkv=2, Hq=8, d=128, n_max=4096, T=16, L_blk=2048, update_interval=1024)
+    K, V, _ = H.cache_for(o, max(n, 1), comps=8, seed=30 + n)
+    oidx = mp.empty_index(o)
+    gidx = MultipoleIndex(H.gcfg(o))
+    if n > 0:
+        assert not mp.cluster_update(oidx, K[:, :, :n], V[:, :, :n])
+        assert not gidx.update(H.tdev(K[:, :, :n], "bf16"), H.tdev(V[:, :, :n], "bf16"))
+    assert gidx.n_tokens == n and gidx.n_clustered == 0
+    Q = synth.make_queries(1, 2, 8, 128, "bf16", seed=n)[0]
+    for budget in (0, 16):
+        O = H.to_np(gidx.decode(H.tdev(Q, "bf16"), budget))
+        torch.cuda.synchronize()
+        assert gidx.check_device_error() == 0
+        O_ref = mp.decode(oidx, Q, budget)
+        assert np.abs(O - O_ref).max() <= H.TOL["bf16"]
+        if n == 0:
+            assert not O.any()

@@ -126,6 +126,23 @@ class MultipoleIndex:
         if tuple(t.shape) != want or t.dtype != c.torch_dtype or not t.is_contiguous() or t.device != self.device:
             raise ValueError(f"expected a contiguous {c.torch_dtype} tensor of shape {want} on {self.device}")
 
+    def _check_q_out(self, Q, out):
+        """Shape, dtype and memory checks of a decode's Q and O; allocates O if absent
+        (pinned host memory for a host Q)."""
+        c = self.cfg
+        want = (c.batch, c.q_heads, c.head_dim)
+        if tuple(Q.shape) != want or Q.dtype != c.torch_dtype or not Q.is_contiguous():
+            raise ValueError(f"Q must be a contiguous {c.torch_dtype} tensor of shape {want}")
+        if Q.device.type == "cpu" and not Q.is_pinned():
+            raise ValueError("a host Q must be in page-locked memory (pin_memory())")
+        if out is None:
+            return torch.empty_like(Q, pin_memory=Q.device.type == "cpu")
+        if (tuple(out.shape) != want or out.dtype != c.torch_dtype or not out.is_contiguous()
+                or (out.device.type == "cpu" and not out.is_pinned())):
+            raise ValueError(f"out must be a contiguous {c.torch_dtype} tensor of shape {want}, "
+                             "on the device or in page-locked host memory")
+        return out
+
     # ------------------------------------------------------------------ calls
     def build(self, K, V, init_centroids=None, stream=None):
         """Cluster K, V [B, Hkv, n, d] from scratch (mp_cluster_build)."""
@@ -182,18 +199,7 @@ class MultipoleIndex:
         scores / coarse_scores (float32 [B, Hkv, slots]).  phase_events: torch.cuda.Event
         objects (already recorded once) that the library records at its kernel boundaries.
         """
-        c = self.cfg
-        want = (c.batch, c.q_heads, c.head_dim)
-        if tuple(Q.shape) != want or Q.dtype != c.torch_dtype or not Q.is_contiguous():
-            raise ValueError(f"Q must be a contiguous {c.torch_dtype} tensor of shape {want}")
-        if Q.device.type == "cpu" and not Q.is_pinned():
-            raise ValueError("a host Q must be in page-locked memory (pin_memory())")
-        if out is None:
-            out = torch.empty_like(Q, pin_memory=Q.device.type == "cpu")
-        elif (tuple(out.shape) != want or out.dtype != c.torch_dtype or not out.is_contiguous()
-              or (out.device.type == "cpu" and not out.is_pinned())):
-            raise ValueError(f"out must be a contiguous {c.torch_dtype} tensor of shape {want}, "
-                             "on the device or in page-locked host memory")
+        out = self._check_q_out(Q, out)
         p = L.MpDecodeParams()
         p.budget = int(budget)
         p.coarse_budget = int(coarse_budget)
@@ -224,12 +230,7 @@ class MultipoleIndex:
         overlap on the GPU race on that array; the first call on a device should
         come before any stream capture.
         """
-        c = self.cfg
-        want = (c.batch, c.q_heads, c.head_dim)
-        if tuple(Q.shape) != want or Q.dtype != c.torch_dtype or not Q.is_contiguous():
-            raise ValueError(f"Q must be a contiguous {c.torch_dtype} tensor of shape {want}")
-        if out is None:
-            out = torch.empty_like(Q)
+        out = self._check_q_out(Q, out)
         p = L.MpDecodeParams()
         p.budget = int(budget)
         p.coarse_budget = int(coarse_budget)

@@ -418,7 +418,94 @@ select_kernel(SelectArgs a) {
   if (need <= 0) mode = 0;
   else if (total <= need) mode = 1;
   else mode = 2;
+  bool resolved = false;
   if (mode == 2) {
+    // First try: 256 bins of equal score width between the smallest and the
+    // largest candidate score (monotone in the score, so the bin where the
+    // weight from the top crosses the budget holds the crossing cluster); if
+    // at most 32 candidates fall in it, one warp sorts them by (key
+    // descending, position ascending) and the crossing one gives (thr_key,
+    // thr_pos).  Otherwise the radix descent below decides.
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int pos = tid; pos < n; pos += kSelThreads)
+      if (s_cnt[pos] > 0) { kmin = min(kmin, s_key[pos]); kmax = max(kmax, s_key[pos]); }
+    kmin = __reduce_min_sync(kFull, kmin);
+    kmax = __reduce_max_sync(kFull, kmax);
+    if (tid % kWarp == 0) { s_warp[tid / kWarp] = (int)kmin; s_hist[tid / kWarp] = (int)kmax; }
+    __syncthreads();
+    kmin = 0xffffffffu; kmax = 0u;
+    for (int w = 0; w < kSelThreads / kWarp; ++w) {
+      kmin = min(kmin, (uint32_t)s_warp[w]);
+      kmax = max(kmax, (uint32_t)s_hist[w]);
+    }
+    __syncthreads();
+    const float smin = key_score(kmin), smax = key_score(kmax);
+    const float span = smax - smin, inv = 256.f / span;
+    if (isfinite(smin) && isfinite(smax) && span > 0.f && isfinite(span) && isfinite(inv)) {
+      auto fbin = [&](uint32_t k) { return min(255, (int)((key_score(k) - smin) * inv)); };
+      if (tid < 256) s_hist[tid] = 0;
+      if (tid == 0) s_bcast[3] = 0;
+      __syncthreads();
+      for (int pos = tid; pos < n; pos += kSelThreads)
+        if (s_cnt[pos] > 0) atomicAdd(&s_hist[fbin(s_key[pos])], s_cnt[pos]);
+      __syncthreads();
+      int v = tid < 256 ? s_hist[255 - tid] : 0;
+      int tot;
+      int before = block_excl_scan<kSelThreads>(v, s_warp, &tot);
+      if (tid < 256 && before < need && before + v >= need) {
+        s_bcast[0] = 255 - tid;
+        s_bcast[1] = before;
+      }
+      __syncthreads();
+      const int fb = s_bcast[0], ab = s_bcast[1];
+      int* lst = s_hist;                                   // [32][3]: the histogram is no longer needed
+      __syncthreads();
+      for (int pos = tid; pos < n; pos += kSelThreads)
+        if (s_cnt[pos] > 0 && fbin(s_key[pos]) == fb) {
+          const int q = atomicAdd(&s_bcast[3], 1);
+          if (q < 32) { lst[3 * q] = (int)s_key[pos]; lst[3 * q + 1] = pos; lst[3 * q + 2] = s_cnt[pos]; }
+        }
+      __syncthreads();
+      const int nc = s_bcast[3];
+      if (nc <= 32) {
+        if (tid < kWarp) {
+          const int lane = tid;
+          uint64_t key = lane < nc ? ((uint64_t)(uint32_t)lst[3 * lane] << 32) |
+                                         (uint32_t)(0xffffffffu - (uint32_t)lst[3 * lane + 1])
+                                   : 0ull;
+          int wl = lane < nc ? lst[3 * lane + 2] : 0;
+#pragma unroll
+          for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+              const uint64_t ok = __shfl_xor_sync(kFull, key, jj);
+              const int ow = __shfl_xor_sync(kFull, wl, jj);
+              const bool up = ((lane & kk) == 0) == ((lane & jj) == 0);   // this lane keeps the larger
+              if (up ? ok > key : ok < key) { key = ok; wl = ow; }
+            }
+          }
+          int inc = wl;
+#pragma unroll
+          for (int o = 1; o < kWarp; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += y;
+          }
+          const unsigned cross = __ballot_sync(kFull, lane < nc && ab + inc >= need);
+          const uint64_t ck = __shfl_sync(kFull, key, __ffs(cross) - 1);
+          if (lane == 0) {
+            s_bcast[0] = (int)(uint32_t)(ck >> 32);
+            s_bcast[2] = (int)(0xffffffffu - (uint32_t)ck);
+          }
+        }
+        __syncthreads();
+        thr_key = (uint32_t)s_bcast[0];
+        thr_pos = s_bcast[2];
+        resolved = true;
+      }
+      __syncthreads();
+    }
+  }
+  if (mode == 2 && !resolved) {
     uint32_t prefix = 0, mask = 0;
     int committed = 0;
     for (int shift = 24; shift >= 0; shift -= 8) {

@@ -147,26 +147,28 @@ def brute_selection(score, count, budget):
     return sel
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("budget", [1, 100, 1124, 3000, 4096, 5000])
-def test_selection_with_exact_score_ties(budget):
+def test_selection_with_exact_score_ties(budget, dtype):
     """The selection as a function of the scores it reports: groups of 64 and of
     4 clusters with identical keys (exact score ties at the crossing, more and
-    fewer candidates than one warp resolves) and one unit of distinct keys."""
-    o = H.ocfg(B=1, Hkv=3, Hq=12, d=128, n_max=4096, T=16, L_blk=4096)
+    fewer candidates than one warp resolves) and one unit of distinct keys;
+    bf16 runs the two-pass kernels, fp32 the multi-kernel path."""
+    o = H.ocfg(B=1, Hkv=3, Hq=12, d=128, n_max=4096, T=16, L_blk=4096, dtype=dtype)
     rng = np.random.default_rng(12)
     K = np.empty((1, 3, 4096, 128), dtype=np.float32)
     for h, grp in enumerate((64, 4, 1)):
-        base = synth._cast(rng.standard_normal((256 // grp, 128)), "bf16")
+        base = synth._cast(rng.standard_normal((256 // grp, 128)), dtype)
         K[0, h] = np.repeat(base, 16 * grp, axis=0)
-    V = synth._cast(rng.standard_normal((1, 3, 4096, 128)), "bf16")
+    V = synth._cast(rng.standard_normal((1, 3, 4096, 128)), dtype)
     a = np.broadcast_to(np.arange(4096) // 16, (1, 3, 4096))
     oidx = mp.index_from_assignment(K, V, 4096, o, a)
     gidx = MultipoleIndex(H.gcfg(o))
     H.upload_index(gidx, oidx)
     mask = torch.zeros((1, 3, gidx.slots), dtype=torch.uint8, device="cuda")
     scores = torch.empty((1, 3, gidx.slots), dtype=torch.float32, device="cuda")
-    Q = synth.make_queries(1, 1, 12, 128, "bf16", seed=6)[0]
-    gidx.decode(H.tdev(Q, "bf16"), budget, sel_mask=mask, scores=scores)
+    Q = synth.make_queries(1, 1, 12, 128, dtype, seed=6)[0]
+    gidx.decode(H.tdev(Q, dtype), budget, sel_mask=mask, scores=scores)
     torch.cuda.synchronize()
     assert gidx.check_device_error() == 0
     count = np.diff(oidx["off"][0], axis=-1)

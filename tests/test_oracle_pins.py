@@ -363,3 +363,24 @@ def test_coarse_centroids_are_means_of_their_tokens():
         assert np.all(np.abs(idx["Kcc"][0, 0, cc] - mean_k) <= tol)
         tolv = 0.5 * np.spacing(np.abs(mean_v).astype(np.float32))
         assert np.all(np.abs(idx["Vcc"][0, 0, cc] - mean_v) <= tolv)
+
+
+@pytest.mark.parametrize("levels", [1, 2])
+def test_output_is_affine_in_the_values(levels):
+    """Softmax weights sum to one and depend on keys only, and centroids are
+    member means: values a*V + b give outputs a*O + b, selection unchanged, for
+    every budget (exact and centroid terms, flat and two-level)."""
+    cfg = ocfg(B=1, Hkv=2, Hq=4, n_max=256, L_blk=128, T=4, Tc=16, levels=levels)
+    K, V, _ = cache(cfg, 256)
+    a, b = 2.0, 0.5 * np.linspace(-1.0, 1.0, cfg["d"])
+    V2 = a * V + b
+    idx1 = mp.build_index(K, V, 256, cfg)
+    idx2 = mp.build_index(K, V2, 256, cfg)
+    Q = synth.make_queries(1, 1, 4, cfg["d"], "f32", seed=13)[0]
+    for budget, cb in [(1, 8), (20, 40), (100, 120), (256, 256)]:
+        i1, i2 = {}, {}
+        O1 = mp.decode(idx1, Q, budget, coarse_budget=cb, info=i1)
+        O2 = mp.decode(idx2, Q, budget, coarse_budget=cb, info=i2)
+        for u in i1:
+            np.testing.assert_array_equal(i1[u]["sel"], i2[u]["sel"])
+        np.testing.assert_allclose(O2, a * O1 + b, atol=1e-6)

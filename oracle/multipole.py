@@ -46,10 +46,11 @@ Readings where the pages are silent (each restated where it is used):
 * R12 k-means++ randomness: splitmix64 (Steele, Lea & Flood, 2014) streams.
 * R13 the online update re-clusters only blocks that hold tail tokens.
 * R14 update init: a block's previous centroids keep their slots; new slots
-      are seeded with the keys of the new tokens at stride T.  Parity
-      unpinned: the pages fix no update initialisation, so only invariants
-      (permutation, member means) and the block-sized case (equal to a fresh
-      stride-seeded build) check it.
+      are seeded with the keys of the new tokens at stride T, counted from the
+      first new token.  The pages fix no update initialisation; this reading
+      is pinned by a hand-worked update of a non-empty block (old slots kept,
+      new seeds at the new tokens) and by the block-sized case (equal to a
+      fresh stride-seeded build).
 * R15 hierarchy: coarse clusters are a count-weighted k-means over a block's
       fine centroids, ceil(L/Tc) of them; fine slots are reordered so every
       coarse cluster owns a contiguous range of fine slots (and of tokens);
@@ -604,7 +605,8 @@ def _scores(q, cents, scale):
     return scale * (q @ cents.T)          # [G, C]
 
 
-def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None):
+def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, force_sel=None,
+           units=None):
     """One decode step for every (batch, query head).  Returns O [B, Hq, d] (fp64).
 
     Flat index (levels == 1), per KV head h and its query heads g (R1):
@@ -618,6 +620,13 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None):
     fine scores and selection only among fine clusters of selected coarse
     clusters, and coarse centroid terms for unselected coarse clusters.
     ``info`` (dict, optional) receives per-unit selections and scores.
+
+    ``force_sel`` (dict, optional): (b, h) -> {"sel": fine cluster ids[,
+    "csel": coarse cluster ids]} replaces the selection step of that unit by the
+    given sets; every other step is unchanged.  Where a score tie (R3) lets more
+    than one set be correct, this gives the output that belongs to a particular
+    one of them.  ``units`` (optional): the (b, h) pairs to compute; the output
+    rows of the other units are left zero.
     """
     cfg = idx["cfg"]
     B, H, Hq, d = cfg["B"], cfg["Hkv"], cfg["Hq"], cfg["d"]
@@ -628,8 +637,12 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None):
         coarse_budget = 8 * budget
     nc, nt = idx["n_clustered"], idx["n_tokens"]
     O = np.zeros((B, Hq, d))
+    todo = None if units is None else {tuple(u) for u in units}
     for b in range(B):
         for h in range(H):
+            if todo is not None and (b, h) not in todo:
+                continue
+            forced = None if force_sel is None else force_sel.get((b, h))
             q = np.asarray(Q[b, h * G:(h + 1) * G], dtype=np.float64)
             off = idx["off"][b, h]
             cnt = counts_of(off)
@@ -640,6 +653,8 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None):
             unit_info = {}
             if cfg.get("levels", 1) == 1:
                 sel, ranked = select_clusters(shat, cnt, budget)
+                if forced is not None:
+                    sel = np.asarray(forced["sel"], dtype=np.int64)
                 approx = np.setdiff1d(np.nonzero(cnt > 0)[0], sel)
                 coarse_terms = np.zeros(0, dtype=np.int64)
                 unit_info.update(sel=sel, ranked=ranked, shat=shat)
@@ -650,12 +665,16 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None):
                 Sc = _scores(q, Kcc, scale)
                 chat = np.where(ccnt > 0, Sc.max(axis=0), -np.inf)
                 csel, cranked = select_clusters(chat, ccnt, coarse_budget)
+                if forced is not None:
+                    csel = np.asarray(forced["csel"], dtype=np.int64)
                 fine_cand = np.zeros(cnt.size, dtype=bool)
                 for cc in csel:
                     fine_cand[coff[cc]:coff[cc + 1]] = True
                 shat_f = np.where(fine_cand & (cnt > 0), shat, -np.inf)
                 cnt_f = np.where(fine_cand, cnt, 0)
                 sel, ranked = select_clusters(shat_f, cnt_f, budget)
+                if forced is not None:
+                    sel = np.asarray(forced["sel"], dtype=np.int64)
                 approx = np.setdiff1d(np.nonzero(cnt_f > 0)[0], sel)
                 coarse_terms = np.setdiff1d(np.nonzero(ccnt > 0)[0], csel)
                 unit_info.update(sel=sel, ranked=ranked, shat=shat_f, csel=csel,
@@ -675,26 +694,6 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None):
             if info is not None:
                 info[(b, h)] = unit_info
     return O
-
-
-def selection_margin(shat, counts, budget):
-    """Smallest score gap that decides the selected set (R2 tie analysis).
-
-    Swapping two clusters inside the selected prefix, or two outside it, does
-    not change the selected set; the set depends only on the order around the
-    crossing cluster.  Returns the smallest |score difference| between the
-    crossing cluster or the last selected cluster and any candidate whose
-    exchange with it changes the set; inf when nothing depends on order.
-    """
-    sel, ranked = select_clusters(shat, counts, budget)
-    if sel.size == 0 or sel.size == ranked.size:
-        return math.inf
-    sel_s = shat[sel]
-    rest_s = shat[ranked[sel.size:]]
-    # any selected cluster within reach of any unselected one can swap places
-    lo = sel_s.min()
-    hi = rest_s.max()
-    return float(abs(lo - hi))
 
 
 def dense_attention(Q, K, V, n, Hkv, scale=None):

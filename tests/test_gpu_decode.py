@@ -36,10 +36,14 @@ def run_decode(o, oidx, Q, budget, coarse_budget=0, no_approx=False, n_split=0, 
     torch.cuda.synchronize()
     assert gidx.check_device_error() == 0
     info = {}
-    O_ref = mp.decode(oidx, Q, budget, coarse_budget=coarse_budget if coarse_budget > 0 else None,
-                      flags=mp.NO_APPROX if no_approx else 0, scale=scale, info=info)
+
+    def oracle(**kw):
+        return mp.decode(oidx, Q, budget, coarse_budget=coarse_budget if coarse_budget > 0 else None,
+                         flags=mp.NO_APPROX if no_approx else 0, scale=scale, **kw)
+    O_ref = oracle(info=info)
     skipped = H.compare_decode(o, H.to_np(O), O_ref, info, mask.cpu().numpy(), scores.cpu().numpy(),
-                               levels=o["levels"], gpu_cmask=None if cmask is None else cmask.cpu().numpy())
+                               levels=o["levels"], gpu_cmask=None if cmask is None else cmask.cpu().numpy(),
+                               redo=lambda fs, units: oracle(force_sel=fs, units=units))
     return skipped, H.to_np(O), O_ref
 
 
@@ -252,9 +256,12 @@ def test_full_size_bench_launch_sampled_units():
     for u in (0, 17, 38, 55, 73, 90, 111, 127):
         b, h = divmod(u, Hkv)
         info = {}
-        O_ref = mp.decode(heads[u % 8], Q[b:b + 1, h * G:(h + 1) * G], w["budget"], info=info)
+        Qu = Q[b:b + 1, h * G:(h + 1) * G]
+        O_ref = mp.decode(heads[u % 8], Qu, w["budget"], info=info)
         skipped += H.compare_decode(o1, O[b:b + 1, h * G:(h + 1) * G], O_ref, info, mask[b:b + 1, h:h + 1],
-                                    scores[b:b + 1, h:h + 1])
+                                    scores[b:b + 1, h:h + 1],
+                                    redo=lambda fs, units, hd=heads[u % 8], q=Qu: mp.decode(hd, q, w["budget"],
+                                                                                           force_sel=fs, units=units))
     assert skipped <= 2
 
 

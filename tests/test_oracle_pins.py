@@ -384,3 +384,135 @@ def test_output_is_affine_in_the_values(levels):
         for u in i1:
             np.testing.assert_array_equal(i1[u]["sel"], i2[u]["sel"])
         np.testing.assert_allclose(O2, a * O1 + b, atol=1e-6)
+
+
+# --------------------------------------------------------------------------- online update, warm start (R14)
+
+def _frac_rows(rows):
+    from fractions import Fraction
+    return np.array([[float(Fraction(x)) for x in r] for r in rows])
+
+
+def _run_warm_start_case(block_init=None):
+    """The hand-worked update of tests/golden/warm_start_update.json through the oracle."""
+    g = json.load(open(os.path.join(GOLD, "warm_start_update.json")))
+    c = g["config"]
+    cfg = ocfg(B=c["B"], Hkv=c["Hkv"], Hq=c["Hq"], d=c["d"], n_max=c["n_max"], T=c["T"], L_blk=c["L_blk"],
+               iters=c["iters"], update_interval=c["update_interval"], dtype=c["dtype"])
+    K = np.array(g["keys"], dtype=np.float64)[None, None]
+    V = np.array(g["values"], dtype=np.float64)[None, None]
+    orig = mp._block_init
+    if block_init is not None:
+        mp._block_init = block_init
+    try:
+        idx = mp.build_index(K, V, 4, cfg, init_mode="stride")
+        built = idx["Kc"][0, 0, :2].copy()
+        rec = []
+        fired = mp.cluster_update(idx, K[:, :, 4:], V[:, :, 4:], record=rec)
+    finally:
+        mp._block_init = orig
+    return g["expected"], built, fired, rec, idx
+
+
+def _matches_warm_start_golden(exp, built, fired, rec, idx):
+    f32 = lambda a: np.asarray(a, dtype=np.float64).astype(np.float32)
+    if not fired or len(rec) != 1:
+        return False
+    b, h, j, _, ini, hist = rec[0]
+    return bool((b, h, j) == (0, 0, 0)
+                and np.array_equal(f32(built), f32(_frac_rows(exp["build_Kc"])))
+                and np.array_equal(f32(ini), f32(_frac_rows(exp["update_init"])))
+                and np.array_equal(hist[0]["assign"], exp["update_assign"])
+                and np.array_equal(f32(idx["Kc"][0, 0]), f32(_frac_rows(exp["Kc"])))
+                and np.array_equal(f32(idx["Vc"][0, 0]), f32(_frac_rows(exp["Vc"])))
+                and np.array_equal(idx["off"][0, 0], exp["off"])
+                and np.array_equal(idx["perm"][0, 0], exp["perm"])
+                and idx["n_clustered"] == 8)
+
+
+def test_warm_start_update_matches_the_hand_worked_case():
+    """R14 with a non-empty previous block: old centroids keep their slots, new
+    slots start at the new tokens' keys at stride T (hand-worked golden)."""
+    assert _matches_warm_start_golden(*_run_warm_start_case())
+
+
+def _slip(kind):
+    """A copy of the oracle's block init with one planted mistake in its warm start."""
+    orig = mp._block_init
+
+    def init(idx, b, h, j, X, L_old, init_mode, unit, init_given):
+        if init_mode != "warm" or L_old == 0:
+            return orig(idx, b, h, j, X, L_old, init_mode, unit, init_given)
+        T = idx["cfg"]["T"]
+        C, C_old = -(-X.shape[0] // T), -(-L_old // T)
+        s0 = j * idx["geom"]["C_blk"]
+        warm = idx["Kc"][b, h, s0:s0 + C_old].copy()
+        if kind == "stride_from_block_start":
+            return np.concatenate([warm, X[T * np.arange(C - C_old)]])
+        if kind == "old_slots_reseeded":
+            return X[T * np.arange(C)]
+        if kind == "stride_one":
+            return np.concatenate([warm, X[L_old + np.arange(C - C_old)]])
+        if kind == "warm_after_new":
+            return np.concatenate([X[L_old + T * np.arange(C - C_old)], warm])
+        raise ValueError(kind)
+    return init
+
+
+@pytest.mark.parametrize("kind", ["stride_from_block_start", "old_slots_reseeded", "stride_one", "warm_after_new"])
+def test_planted_warm_start_slips_fail_the_hand_worked_case(kind):
+    """Each plausible mistake in the warm start, planted in the oracle, fails the golden case."""
+    assert not _matches_warm_start_golden(*_run_warm_start_case(_slip(kind)))
+
+
+# --------------------------------------------------------------------------- dense attention checker
+
+@pytest.mark.parametrize("Hkv,Hq", [(2, 2), (2, 8), (3, 12)])
+def test_dense_attention_equals_torch_sdpa(Hkv, Hq):
+    """The dense checker (GQA: query head g reads KV head g // G) against torch's
+    fp64 SDPA over the first n of more keys; keys, values and queries per head differ."""
+    rng = np.random.default_rng(Hq)
+    B, n_all, n, d = 2, 40, 33, 16
+    K = rng.standard_normal((B, Hkv, n_all, d))
+    V = rng.standard_normal((B, Hkv, n_all, d))
+    Q = 2.0 * rng.standard_normal((B, Hq, d))
+    np.testing.assert_allclose(mp.dense_attention(Q, K, V, n, Hkv), sdpa(Q, K, V, n, Hkv), atol=1e-12)
+    np.testing.assert_allclose(mp.dense_attention(Q, K, V, n, Hkv, scale=0.3), sdpa(Q, K, V, n, Hkv, scale=0.3),
+                               atol=1e-12)
+
+
+# --------------------------------------------------------------------------- forced selections
+
+@pytest.mark.parametrize("levels", [1, 2])
+def test_forcing_the_natural_selection_changes_nothing(levels):
+    """decode(force_sel=its own selection) is bit-identical, unit by unit."""
+    cfg = ocfg(B=2, Hkv=2, Hq=4, n_max=256, L_blk=64, T=4, levels=levels, Tc=16)
+    K, V, _ = cache(cfg, 256)
+    idx = mp.build_index(K, V, 256, cfg)
+    Q = synth.make_queries(1, 2, 4, cfg["d"], "f32", seed=3)[0]
+    info = {}
+    O = mp.decode(idx, Q, 30, coarse_budget=90, info=info)
+    force = {u: {"sel": i["sel"], "csel": i.get("csel")} for u, i in info.items()}
+    np.testing.assert_array_equal(mp.decode(idx, Q, 30, coarse_budget=90, force_sel=force), O)
+    part = mp.decode(idx, Q, 30, coarse_budget=90, units=[(1, 0)])
+    np.testing.assert_array_equal(part[1, 0:2], O[1, 0:2])
+    assert not part[0].any() and not part[1, 2:].any()
+
+
+def test_forcing_every_cluster_is_dense_and_forcing_none_is_all_centroids():
+    """A forced set replaces only the selection: all clusters gives dense
+    attention; no cluster gives the softmax over every centroid term."""
+    cfg = ocfg(B=1, Hkv=1, Hq=4, n_max=128, L_blk=64, T=4)
+    K, V, _ = cache(cfg, 128)
+    idx = mp.build_index(K, V, 128, cfg)
+    Q = synth.make_queries(1, 1, 4, cfg["d"], "f32", seed=4)[0]
+    cnt = mp.counts_of(idx["off"][0, 0])
+    nz = np.nonzero(cnt > 0)[0]
+    O_all = mp.decode(idx, Q, 1, force_sel={(0, 0): {"sel": nz}})
+    np.testing.assert_allclose(O_all, sdpa(Q, K, V, 128, 1), atol=1e-12)
+    O_none = mp.decode(idx, Q, 1, force_sel={(0, 0): {"sel": np.zeros(0, dtype=np.int64)}})
+    Kc, Vc = idx["Kc"][0, 0][nz], idx["Vc"][0, 0][nz]
+    for g in range(4):
+        z = (Kc @ Q[0, g]) / math.sqrt(cfg["d"]) + np.log(cnt[nz])
+        p = np.exp(z - z.max())
+        np.testing.assert_allclose(O_none[0, g], p @ Vc / p.sum(), atol=1e-12)

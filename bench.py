@@ -284,7 +284,9 @@ def run_ours(args, w):
     if idx.check_device_error() != 0:
         raise RuntimeError("device error after build")
     kassign = time_assign(idx, Kd, w, args) if not args.no_assign else None
-    del Kd, Vd
+    if args.no_extras or world > 1:
+        del Kd, Vd
+        Kd = Vd = None
     nq = args.warmup + args.steps
     Qh = synth.make_queries(nq, B, Hq, d, w["dtype"], seed=w["seed"] + 7 + 100 * rank)
     Q = torch.from_numpy(Qh).to(dev).to(tdt)
@@ -378,7 +380,7 @@ def run_ours(args, w):
     C_tot = int(C_unit.sum())
     sel_tot = sum(step_bytes) / len(step_bytes)
     phase_alg = {
-        "centroid pass + value pass": sel_tot,
+        "decode": sel_tot,
         "centroid pass": 2 * C_tot * d * e + (idx.slots + 1) * 4 * B * Hkv,
         "token pass": sel_tot - (2 * C_tot * d * e + (idx.slots + 1) * 4 * B * Hkv) - 2 * B * Hq * d * e,
     }
@@ -390,6 +392,11 @@ def run_ours(args, w):
         roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(dom_name, args.workload),
                 "kernel": dom_name, "peak_source": pk["source"]}
+
+    extras = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        extras = run_extras(args, w, dev, cfg, Kd, Vd, Qh, 1e3 * ms_per_step)
+        del Kd, Vd
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -414,17 +421,171 @@ def run_ours(args, w):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_bytes / e2e_time / 1e9, "unit": UNIT, "h2d_bytes_per_step": qbytes,
                     "d2h_bytes_per_step": qbytes},
-            "gpu_launches": args.steps * (2 if names[-1] == "centroid pass + value pass" else len(names)),
+            "gpu_launches": args.steps * len(names),
             "clocks": clk,
             "build_s": build_s,
             "kmeans_assign": kassign,
             "selected_tokens_per_head": sel_tokens_mean,
+            "extra_configs": extras,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+# ----------------------------------------------------------------------------- other configurations
+def make_flusher(dev):
+    """write 2x L2, then read another 2x L2: the next step starts from a cold, clean L2"""
+    import torch
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
+    fw = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    fr = torch.ones(2 * l2, dtype=torch.uint8, device=dev)
+
+    def flush():
+        fw.zero_()
+        fr.amax()
+    return flush
+
+
+def time_steps(fn, steps, warmup, flush):
+    """Device time (ms) of `steps` calls fn(i) after `warmup` untimed ones, L2 flushed before each
+    (outside the events), CUDA events on the launching stream."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        flush()
+        fn(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        ev[i][0].record(stream)
+        fn(warmup + i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def hier_bytes_unit(w, cc_nonempty, n_cand, n_sel_tokens):
+    """Bytes one two-level (batch, KV head) step must read or write: every coarse key and value
+    centroid and coarse range, the key and value centroids and offsets of the fine clusters inside
+    the selected coarse clusters, the selected tokens' keys and values, Q and O."""
+    e = 2 if w["dtype"] == "bf16" else 4
+    d, G = w["d"], w["Hq"] // w["Hkv"]
+    return (2 * cc_nonempty * d * e + (cc_nonempty + 1) * 4 + 2 * n_cand * d * e + (n_cand + 1) * 4
+            + 2 * n_sel_tokens * d * e + 2 * G * d * e)
+
+
+def run_extra_decode(name, args, dev, pk, flush):
+    """Decode µs/step of another configuration (its own cache, build and queries)."""
+    import torch
+    from clustered_sparse_decode_b200 import Config, MultipoleIndex, synth
+    w = synth.workload(name)
+    B, Hkv, Hq, d, n = w["B"], w["Hkv"], w["Hq"], w["d"], w["n"]
+    tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+    K, V, _ = synth.make_cache(B, Hkv, n, d, w["comps"], w["sigma"], radius=w["radius"], outliers=w["outliers"],
+                               dtype=w["dtype"], seed=w["seed"])
+    Kd, Vd = torch.from_numpy(K).to(dev).to(tdt), torch.from_numpy(V).to(dev).to(tdt)
+    del K, V
+    levels = w.get("levels", 1)
+    cfg = Config(batch=B, kv_heads=Hkv, q_heads=Hq, head_dim=d, max_tokens=n, tokens_per_centroid=w["T"],
+                 block_tokens=w["L_blk"], levels=levels, coarse_tokens_per_centroid=w.get("Tc", 128),
+                 kmeans_iters=w["iters"], dtype=w["dtype"], seed=w["seed"])
+    idx = MultipoleIndex(cfg, device=dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    idx.build(Kd, Vd)
+    torch.cuda.synchronize()
+    build_s = time.perf_counter() - t0
+    del Kd, Vd
+    if idx.check_device_error() != 0:
+        raise RuntimeError(f"device error after the {name} build")
+    steps = min(args.steps, 20)
+    Qh = synth.make_queries(args.warmup + steps, B, Hq, d, w["dtype"], seed=w["seed"] + 7)
+    Q = torch.from_numpy(Qh).to(dev).to(tdt)
+    O = torch.empty((B, Hq, d), dtype=tdt, device=dev)
+    budget, cb = w["budget"], w.get("coarse_budget", 0)
+    # algorithmic bytes of every timed step, from its own selection (untimed pass)
+    arr = idx.arrays()
+    off = arr["off"].to(torch.int64)
+    cnt = off[:, :, 1:] - off[:, :, :-1]
+    mask = torch.zeros((B, Hkv, idx.slots), dtype=torch.uint8, device=dev)
+    cmask = torch.zeros((B, Hkv, max(idx.coarse_slots, 1)), dtype=torch.uint8, device=dev) if levels == 2 else None
+    step_bytes = []
+    for i in range(args.warmup, args.warmup + steps):
+        idx.decode(Q[i], budget, coarse_budget=cb, out=O, sel_mask=mask, coarse_sel_mask=cmask)
+        nsel = (cnt * mask.to(torch.int64)).sum(dim=2)
+        tot = 0
+        if levels == 1:
+            C_unit = (cnt > 0).sum(dim=2)
+            for b in range(B):
+                for h in range(Hkv):
+                    tot += algorithmic_bytes_unit(w, int(C_unit[b, h]), int(nsel[b, h]), 0)
+        else:
+            coff = arr["coff"].to(torch.int64)
+            ccnt = off.gather(2, coff[:, :, 1:]) - off.gather(2, coff[:, :, :-1])
+            cc_ne = (ccnt > 0).sum(dim=2)
+            for b in range(B):
+                for h in range(Hkv):
+                    cand = 0
+                    for c in torch.nonzero(cmask[b, h]).flatten().tolist():
+                        r0, r1 = int(coff[b, h, c]), int(coff[b, h, c + 1])
+                        cand += int((cnt[b, h, r0:r1] > 0).sum())
+                    tot += hier_bytes_unit(w, int(cc_ne[b, h]), cand, int(nsel[b, h]))
+        step_bytes.append(tot)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_steps(lambda i: idx.decode(Q[i], budget, coarse_budget=cb, out=O), steps, args.warmup, flush)
+    clk = clocks.stop()
+    if idx.check_device_error() != 0:
+        raise RuntimeError(f"device error in the {name} decode")
+    us = 1e3 * statistics.mean(ms)
+    gbs = sum(step_bytes) / (sum(ms) / 1e3) / 1e9
+    return {"us_per_step": us, "gb_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "tokens_per_s": B * 1e6 / us,
+            "bytes_per_step": statistics.mean(step_bytes), "build_s": build_s, "steps": steps,
+            "budget": budget, "coarse_budget": cb if levels == 2 else None, "clocks": clk,
+            "config": {"batch": B, "kv_heads": Hkv, "q_heads": Hq, "head_dim": d, "context": n, "levels": levels}}
+
+
+def run_extras(args, w, dev, cfg, Kd, Vd, Qh, us_headline):
+    """The other configurations, each with its own clock record: the dense decode baseline on the
+    headline's cache, single-sequence 32K, two-level 64K, and the online workload."""
+    import torch
+    from clustered_sparse_decode_b200 import dense_decode
+    pk = peaks()
+    flush = make_flusher(dev)
+    out = {}
+    # dense baseline: every key of the same cache, exact (a FlashDecoding-style split-KV decode)
+    tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+    Q = torch.from_numpy(Qh).to(dev).to(tdt)
+    O = torch.empty_like(Q[0])
+    steps = min(args.steps, 20)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_steps(lambda i: dense_decode(cfg, Kd, Vd, w["n"], Q[i % Q.shape[0]], out=O), steps, args.warmup, flush)
+    clk = clocks.stop()
+    e = 2 if w["dtype"] == "bf16" else 4
+    dense_bytes = w["B"] * w["Hkv"] * w["n"] * w["d"] * 2 * e + 2 * w["B"] * w["Hq"] * w["d"] * e
+    us = 1e3 * statistics.mean(ms)
+    gbs = dense_bytes / (us / 1e6) / 1e9
+    out["dense_baseline"] = {"us_per_step": us, "gb_s": gbs, "frac_hbm": gbs / pk["hbm_gbs"],
+                             "bytes_per_step": dense_bytes, "multipole_speedup": us / us_headline, "clocks": clk,
+                             "what": "exact attention over all keys of the same cache (mp_dense_decode)"}
+    del Q, O
+    for name in ("single_bf16", "hier_64k"):
+        out[name] = run_extra_decode(name, args, dev, pk, flush)
+    ow = synth_workload("online_16k_plus_16k")
+    out["online_16k_plus_16k"] = online_measure(args, ow, dev, 0, 1, None)
+    return out
+
+
+def synth_workload(name):
+    from clustered_sparse_decode_b200 import synth
+    return synth.workload(name)
 
 
 def run_online(args, w):
@@ -436,7 +597,6 @@ def run_online(args, w):
     import torch
     import torch.distributed as dist
 
-    from clustered_sparse_decode_b200 import Config, MultipoleIndex, synth
     from clustered_sparse_decode_b200 import build as libbuild
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -448,6 +608,35 @@ def run_online(args, w):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
     libbuild.build()
     dev = torch.device("cuda", local)
+    r = online_measure(args, w, dev, rank, world, dist if world > 1 else None)
+    if rank == 0:
+        line = {
+            "metric": "online decode + amortised cluster update, us per generated token", "value": r["us_per_token"],
+            "unit": "us/token", "n_gpus": world, "steps": r["generated"], "warmup": args.warmup,
+            "ms_per_step": r["us_per_token"] / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+            "config": {"workload": args.workload, "batch": w["B"], "kv_heads": w["Hkv"], "q_heads": w["Hq"],
+                       "head_dim": w["d"], "prompt": w["n"], "generated": r["generated"], "budget": w["budget"],
+                       "block_tokens": w["L_blk"], "update_interval": w["update_interval"],
+                       "kmeans_iters": w["iters"],
+                       "l2": "flushed before every generated token (2x L2 written, then 2x L2 read)",
+                       "parallelism": f"dp{world} (independent batches)"},
+        }
+        line.update({k: v for k, v in r.items() if k not in ("generated",)})
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def online_measure(args, w, dev, rank, world, dist):
+    """Per generated token: mp_cluster_update (append; re-cluster the open block on a
+    trigger) and one decode step, each bracketed by CUDA events, L2 flushed before each
+    token outside the events.  Returns the per-token times (max over ranks)."""
+    import torch
+
+    from clustered_sparse_decode_b200 import Config, MultipoleIndex, synth
     B, Hkv, Hq, d, n0, ng = w["B"], w["Hkv"], w["Hq"], w["d"], w["n"], w["n_gen"]
     if args.gen_tokens > 0:
         ng = min(ng, args.gen_tokens)
@@ -469,26 +658,22 @@ def run_online(args, w):
     Qh = synth.make_queries(args.warmup + ng, B, Hq, d, w["dtype"], seed=w["seed"] + 7 + 100 * rank)
     Q = torch.from_numpy(Qh).to(dev).to(tdt)
     O = torch.empty((B, Hq, d), dtype=tdt, device=dev)
-    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20)
-    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-    flush_r = torch.ones(2 * l2, dtype=torch.uint8, device=dev)
+    flush = make_flusher(dev)
     stream = torch.cuda.current_stream()
     for s in range(args.warmup):
-        flush_w.zero_()
-        flush_r.amax()
+        flush()
         idx.decode(Q[s], w["budget"], out=O)
     torch.cuda.synchronize()
-    if world > 1:
+    if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
     time.sleep(0.3)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(ng)]
     fired = []
     for t in range(ng):
-        flush_w.zero_()
-        flush_r.amax()
+        flush()
         e = ev[t]
         e[0].record(stream)
         fired.append(idx.update(Kgen[t].unsqueeze(2), Vgen[t].unsqueeze(2)))
@@ -496,7 +681,7 @@ def run_online(args, w):
         idx.decode(Q[args.warmup + t], w["budget"], out=O)
         e[2].record(stream)
     torch.cuda.synchronize()
-    if world > 1:
+    if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -508,28 +693,11 @@ def run_online(args, w):
     fired_ms = sum(u for u, f in zip(upd, fired) if f)
     dec_ms = sum(ev[t][1].elapsed_time(ev[t][2]) for t in range(ng))
     tot_tokens, tot_s = aggregate(B * ng, (upd_ms + dec_ms) / 1e3, dist)
-    us_per_token = 1e6 * tot_s / ng
-    if rank == 0:
-        line = {
-            "metric": "online decode + amortised cluster update, us per generated token", "value": us_per_token,
-            "unit": "us/token", "n_gpus": world, "steps": ng, "warmup": args.warmup,
-            "ms_per_step": us_per_token / 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-            "dtype": w["dtype"], "data": "synthetic",
-            "config": {"workload": args.workload, "batch": B, "kv_heads": Hkv, "q_heads": Hq, "head_dim": d,
-                       "prompt": n0, "generated": ng, "budget": w["budget"], "block_tokens": w["L_blk"],
-                       "update_interval": w["update_interval"], "kmeans_iters": w["iters"],
-                       "l2": "flushed before every generated token (2x L2 written, then 2x L2 read)",
-                       "parallelism": f"dp{world} (independent batches)"},
+    return {"us_per_token": 1e6 * tot_s / ng, "generated": ng,
             "decode_us_per_token": 1e3 * dec_ms / ng, "update_us_per_token": 1e3 * upd_ms / ng,
             "reclusterings": n_fired, "recluster_ms_each": fired_ms / max(n_fired, 1),
             "append_us_each": 1e3 * (upd_ms - fired_ms) / max(ng - n_fired, 1), "tokens_per_s": tot_tokens / tot_s,
-            "clocks": clk,
-        }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+            "clocks": clk}
 
 
 def assign_flops(w):
@@ -589,7 +757,7 @@ def traffic_for(kernel, workload):
 
 
 # the sources of each kernel whose traffic profiles/traffic.md records
-KERNEL_SOURCES = {"centroid pass + value pass": ("decode_stream.cu", "mp_internal.cuh")}
+KERNEL_SOURCES = {"decode": ("decode_unit.cu", "stream_common.cuh", "mp_internal.cuh")}
 
 
 def source_digest(kernel=None):
@@ -614,6 +782,8 @@ def main(argv=None):
     ap.add_argument("--ref-seconds-per-step", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-assign", action="store_true", help="skip the timed k-means assignment step")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations (dense baseline, single sequence, two-level, online)")
     ap.add_argument("--gen-tokens", type=int, default=0,
                     help="online workloads: generated tokens to time (0 = all of the workload's)")
     args = ap.parse_args(argv)

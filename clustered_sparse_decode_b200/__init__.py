@@ -6,5 +6,5 @@ attends exactly to the top clusters up to a token budget and approximates the
 rest by count-weighted centroid terms.  The work runs in the CUDA library
 libmpattn.so (C ABI in include/mpattn.h); this package is its Python binding.
 """
-from .api import Config, MultipoleIndex, workspace_size  # noqa: F401
+from .api import Config, MultipoleIndex, dense_decode, workspace_size  # noqa: F401
 from ._lib import MpError  # noqa: F401

@@ -10,12 +10,11 @@ MP_F32, MP_BF16 = 0, 1
 MP_INIT_KMEANSPP, MP_INIT_STRIDE = 0, 1
 MP_NO_APPROX = 1
 MP_STATIC_SCRATCH_BYTES = 32 << 20
-MP_SCRATCH_TICKET_BYTES = 4096
 
 EXPORTS = ["mp_workspace_size", "mp_index_init", "mp_cluster_build", "mp_cluster_update", "mp_cluster_assign",
-           "mp_decode",
-           "mp_decode_static", "mp_decode_static_reset",
-           "mp_index_export", "mp_index_import", "mp_check_device_error", "mp_status_str"]
+           "mp_decode", "mp_dense_decode",
+           "mp_decode_static",
+           "mp_index_export", "mp_index_import", "mp_check_device_error", "mp_decode_phases", "mp_status_str"]
 
 
 class MpConfig(ctypes.Structure):
@@ -77,7 +76,7 @@ def load():
         "mp_cluster_assign": [P(MpIndex), vp, i32, vp, vp],
         "mp_decode": [P(MpIndex), vp, vp, P(MpDecodeParams), vp, sz, vp],
         "mp_decode_static": [P(MpIndex), vp, vp, P(MpDecodeParams), vp],
-        "mp_decode_static_reset": [vp],
+        "mp_dense_decode": [P(MpConfig), vp, vp, i32, vp, vp, ctypes.c_float, vp],
         "mp_index_export": [P(MpIndex), P(MpIndexView)],
         "mp_index_import": [P(MpIndex), P(MpIndexView), i64, i64, vp],
         "mp_check_device_error": [P(MpIndex), P(i32), vp],
@@ -86,6 +85,8 @@ def load():
         f = getattr(lib, name)
         f.argtypes = args
         f.restype = ctypes.c_int
+    lib.mp_decode_phases.argtypes = [P(MpIndex)]
+    lib.mp_decode_phases.restype = ctypes.c_char_p
     lib.mp_status_str.argtypes = [ctypes.c_int]
     lib.mp_status_str.restype = ctypes.c_char_p
     _lib = lib

@@ -69,6 +69,28 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
+def dense_decode(cfg: Config, K, V, n, Q, out=None, scale=0.0, stream=None):
+    """Exact attention of every query head over keys [0, n) of its KV head (mp_dense_decode).
+
+    K, V: contiguous device tensors [B, Hkv, max_tokens, d]; Q: [B, Hq, d]; returns
+    O [B, Hq, d].  The dense comparison point of the method, on the same engine.
+    """
+    lib = L.load()
+    want = (cfg.batch, cfg.kv_heads, cfg.max_tokens, cfg.head_dim)
+    for t in (K, V):
+        if tuple(t.shape) != want or t.dtype != cfg.torch_dtype or not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError(f"K and V must be contiguous {cfg.torch_dtype} device tensors of shape {want}")
+    qw = (cfg.batch, cfg.q_heads, cfg.head_dim)
+    if tuple(Q.shape) != qw or Q.dtype != cfg.torch_dtype or not Q.is_contiguous() or Q.device.type != "cuda":
+        raise ValueError(f"Q must be a contiguous {cfg.torch_dtype} device tensor of shape {qw}")
+    if out is None:
+        out = torch.empty_like(Q)
+    c = cfg.to_c()
+    L.check(lib.mp_dense_decode(ctypes.byref(c), _ptr(K), _ptr(V), int(n), _ptr(Q), _ptr(out), float(scale),
+                                _stream(stream)), "mp_dense_decode")
+    return out
+
+
 class MultipoleIndex:
     """Clustered KV cache of one attention layer: build, update, decode."""
 
@@ -79,8 +101,8 @@ class MultipoleIndex:
         ib, sb = workspace_size(cfg)
         with torch.cuda.device(self.device):
             self.workspace = torch.empty(ib, dtype=torch.uint8, device=self.device)
-            # zeroed once: mp_decode keeps the scratch's ticket head zero between steps
-            self.scratch = torch.zeros(sb, dtype=torch.uint8, device=self.device)
+            self.scratch_bytes = sb
+            self._scratch = None     # allocated by the first decode() (decode_static() needs none)
             self.h = L.MpIndex()
             c = cfg.to_c()
             L.check(self.lib.mp_index_init(ctypes.byref(c), _ptr(self.workspace), ib, ctypes.byref(self.h),
@@ -104,21 +126,9 @@ class MultipoleIndex:
         return self.h.coarse_slots
 
     def decode_phases(self):
-        """Names of the intervals between the phase events that decode() records for this index.
-
-        A flat bf16 index with at most 4096 slots per unit, fewer than 512
-        units and at least 8 tokens decodes with a centroid pass and a value
-        pass; the others run a longer kernel pipeline.
-        """
-        c = self.cfg
-        units = c.batch * c.kv_heads
-        if (c.levels == 1 and c.dtype == "bf16" and c.head_dim in (64, 128) and self.slots <= 4096
-                and units < 512 and self.n_tokens >= 8 and c.max_tokens <= (1 << 25)
-                and units * c.max_tokens < 2 ** 31 - 1 and c.q_heads // c.kv_heads in (1, 2, 4, 8)):
-            return ["centroid pass + value pass"]
-        if c.levels == 1:
-            return ["centroid pass", "select", "token pass", "combine"]
-        return ["coarse pass", "coarse select", "fine pass", "fine select", "token pass", "combine"]
+        """Names of the intervals between the phase events that decode() records
+        for this index, as the library reports them (mp_decode_phases)."""
+        return self.lib.mp_decode_phases(ctypes.byref(self.h)).decode().split("|")
 
     def _check_kv(self, t, n):
         c = self.cfg
@@ -282,19 +292,18 @@ class MultipoleIndex:
         L.check(self.lib.mp_index_import(ctypes.byref(self.h), ctypes.byref(v), int(n_tokens), int(n_clustered),
                                          _stream(stream)), "mp_index_import")
 
-    def check_device_error(self, stream=None):
-        """Synchronise and return the device error word (0 = none); clears it.
+    @property
+    def scratch(self):
+        """The decode scratch of mp_decode (device bytes), allocated on first use."""
+        if self._scratch is None:
+            with torch.cuda.device(self.device):
+                self._scratch = torch.empty(self.scratch_bytes, dtype=torch.uint8, device=self.device)
+        return self._scratch
 
-        After an error the ticket heads of this index's decode scratch and of
-        the library's own scratch are zeroed again (a step that stopped early
-        may have left arrival counters behind)."""
+    def check_device_error(self, stream=None):
+        """Synchronise and return the device error word (0 = none); clears it."""
         code = ctypes.c_int32(0)
         st = self.lib.mp_check_device_error(ctypes.byref(self.h), ctypes.byref(code), _stream(stream))
         if st not in (L.MP_OK, L.MP_EDEVICE):
             L.check(st, "mp_check_device_error")
-        if code.value != 0:
-            with torch.cuda.device(self.device):
-                self.scratch[:L.MP_SCRATCH_TICKET_BYTES].zero_()
-                L.check(self.lib.mp_decode_static_reset(_stream(stream)), "mp_decode_static_reset")
-                torch.cuda.synchronize(self.device)
         return code.value

@@ -12,7 +12,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmpattn.so")
-SOURCES = ["api.cu", "assign_tc.cu", "decode.cu", "decode_static.cu", "decode_stream.cu", "kmeans.cu"]
+SOURCES = ["api.cu", "assign_tc.cu", "decode.cu", "decode_static.cu", "decode_unit.cu", "kmeans.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "--shared"]
 

@@ -10,9 +10,12 @@ mp_status build_impl(mp_index* idx, const void* K, const void* V, int32_t n, con
 mp_status update_impl(mp_index* idx, const void* K_new, const void* V_new, int32_t n_new, int32_t* fired,
                       cudaStream_t st);
 mp_status assign_impl(const mp_index* idx, const void* K, int32_t n, int32_t* out, cudaStream_t st);
+const char* decode_phase_names(const mp_index* idx);
 mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
                       size_t scratch_bytes, cudaStream_t st);
 size_t decode_scratch_bytes(const mp_config& c, int slots, int coarse_slots);
+mp_status dense_decode_impl(const mp_config& c, const void* K, const void* V, int n, const void* Q, void* O,
+                            float scale, cudaStream_t st);
 
 int elem_bytes(int dtype) { return dtype == MP_BF16 ? 2 : 4; }
 
@@ -190,6 +193,20 @@ mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode
   return decode_impl(idx, Q, O, p, d_scratch, scratch_bytes, static_cast<cudaStream_t>(stream));
 }
 
+mp_status mp_dense_decode(const mp_config* c, const void* K, const void* V, int32_t n, const void* Q, void* O,
+                          float scale, void* stream) {
+  if (!c || !K || !V || !Q || !O || !std::isfinite(scale)) return MP_EINVAL;
+  if (c->batch < 1 || c->kv_heads < 1 || c->q_heads < 1 || c->q_heads % c->kv_heads != 0 || c->max_tokens < 1)
+    return MP_EINVAL;
+  if (n < 0 || n > c->max_tokens) return MP_EINVAL;
+  if (c->dtype != MP_F32 && c->dtype != MP_BF16) return MP_EINVAL;
+  const int G = c->q_heads / c->kv_heads;
+  if (c->dtype != MP_BF16 || (c->head_dim != 64 && c->head_dim != 128) || (G != 1 && G != 2 && G != 4 && G != 8))
+    return MP_EUNSUPPORTED;
+  if ((int64_t)c->batch * c->kv_heads * c->max_tokens + 64 >= (int64_t)INT32_MAX) return MP_EUNSUPPORTED;
+  return dense_decode_impl(*c, K, V, n, Q, O, scale, static_cast<cudaStream_t>(stream));
+}
+
 mp_status mp_index_export(const mp_index* idx, mp_index_view* v) {
   if (!idx || !idx->workspace || !v) return MP_EINVAL;
   v->Kc = ws_ptr(idx, S_KC);
@@ -259,6 +276,11 @@ mp_status mp_check_device_error(const mp_index* idx, int32_t* code, void* stream
     return MP_EDEVICE;
   }
   return MP_OK;
+}
+
+const char* mp_decode_phases(const mp_index* idx) {
+  if (!idx) return "";
+  return decode_phase_names(idx);
 }
 
 const char* mp_status_str(mp_status s) {

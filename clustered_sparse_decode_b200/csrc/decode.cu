@@ -718,7 +718,7 @@ static DecodeLayout decode_layout(const mp_config& c, int slots, int coarse_slot
   L.cap_fine = coarse_slots;
   L.cap_sub = slots;
   L.cap_csub = coarse_slots;
-  size_t cur = kScratchTicketBytes;   // the two-pass decode's ticket words stay untouched
+  size_t cur = 0;
   const size_t rows = (size_t)L.units * L.G;
   L.o_pm = cur; cur = align256(cur + rows * L.P * 4);
   L.o_pl = cur; cur = align256(cur + rows * L.P * 4);
@@ -735,16 +735,17 @@ static DecodeLayout decode_layout(const mp_config& c, int slots, int coarse_slot
   return L;
 }
 
-size_t stream_scratch_bytes(const mp_config& c, int slots);
-bool stream_supported(const mp_config& c, int slots, int64_t n_tokens);
-mp_status stream_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
-                        size_t scratch_bytes, float scale, cudaStream_t st);
+size_t unit_scratch_bytes(const mp_config& c, int slots);
+bool unit_supported(const mp_config& c, int slots);
+mp_status unit_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
+                      size_t scratch_bytes, float scale, cudaStream_t st);
 
-// Both decode paths place their scratch from the start of the buffer (one call
-// uses one of them); after them, room for a device copy of Q when the caller's
-// Q is page-locked host memory.
+// The decode path of an index places its scratch from the start of the
+// buffer; after it, room for a device copy of Q when the caller's Q is
+// page-locked host memory.
 static size_t q_stage_offset(const mp_config& c, int slots, int coarse_slots) {
-  return align256(std::max(decode_layout(c, slots, coarse_slots).bytes, stream_scratch_bytes(c, slots)));
+  if (unit_supported(c, slots)) return align256(unit_scratch_bytes(c, slots));
+  return align256(decode_layout(c, slots, coarse_slots).bytes);
 }
 static size_t q_bytes(const mp_config& c) {
   return (size_t)c.batch * c.q_heads * c.head_dim * elem_bytes(c.dtype);
@@ -848,6 +849,14 @@ static void record_phase(const mp_decode_params* prm, int i, cudaStream_t st) {
 static mp_status decode_paths(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
                               void* scratch, size_t scratch_bytes, cudaStream_t st);
 
+// Names of the intervals between the phase events of a decode of this index.
+const char* decode_phase_names(const mp_index* idx) {
+  const mp_config& c = idx->cfg;
+  if (unit_supported(c, idx->slots)) return "decode";
+  if (c.levels == 1) return "centroid pass|select|token pass|combine";
+  return "coarse pass|coarse select|fine pass|fine select|token pass|combine";
+}
+
 mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
                       void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const mp_config& c = idx->cfg;
@@ -876,10 +885,10 @@ mp_status decode_impl(const mp_index* idx, const void* Q, void* O, const mp_deco
 static mp_status decode_paths(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm,
                               void* scratch, size_t scratch_bytes, cudaStream_t st) {
   const mp_config& c = idx->cfg;
-  // flat bf16 index: the one-kernel streaming path (decode_stream.cu)
-  if (stream_supported(c, idx->slots, idx->n_tokens)) {
+  // flat bf16 index: one kernel, one CTA (or CTA cluster) per unit (decode_unit.cu)
+  if (unit_supported(c, idx->slots)) {
     const float sc = prm->scale != 0.f ? prm->scale : 1.0f / sqrtf((float)c.head_dim);
-    return stream_decode(idx, Q, O, prm, scratch, scratch_bytes, sc, st);
+    return unit_decode(idx, Q, O, prm, scratch, scratch_bytes, sc, st);
   }
   DecodeLayout L = decode_layout(c, idx->slots, idx->coarse_slots);
   if (scratch_bytes < L.bytes) return MP_ENOSPC;

@@ -22,18 +22,43 @@ size_t decode_scratch_bytes(const mp_config& c, int slots, int coarse_slots);
 // symbol, never a device address: the address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_decode_scratch[MP_STATIC_SCRATCH_BYTES];
 
+// The array's device address belongs to the module loaded in one CUDA
+// context: it is looked up again whenever the device's current context is not
+// the one it was looked up in (after cudaDeviceReset, or when the caller made
+// another driver-API context current).
 constexpr int kMaxDevices = 64;
 static std::mutex g_scratch_mu;
-static void* g_scratch_addr[kMaxDevices];   // device address of g_decode_scratch, per device
+static void* g_scratch_addr[kMaxDevices];   // device address of g_decode_scratch, per device ...
+static void* g_scratch_ctx[kMaxDevices];    // ... in this context
 
-// Device address of the scratch on the current device; resolved on first use.
+using CtxGetCurrent = int (*)(void**);       // cuCtxGetCurrent(CUcontext*) of the driver API
+static CtxGetCurrent ctx_get_current() {
+  static CtxGetCurrent fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrent>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch on the current device and context.
 static mp_status scratch_address(int dev, void** out) {
   if (dev < 0 || dev >= kMaxDevices) return MP_EUNSUPPORTED;
+  CtxGetCurrent get = ctx_get_current();
+  void* ctx = nullptr;
+  if (!get || get(&ctx) != 0) return MP_ECUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!ctx || !g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
+    // the lookup also makes the runtime's context current if none was
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return MP_ECUDA;
+    if (!ctx && (get(&ctx) != 0 || !ctx)) return MP_ECUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_addr[dev];
   return MP_OK;
@@ -59,18 +84,7 @@ extern "C" mp_status mp_decode_static(const mp_index* idx, const void* Q, void* 
   void* scratch = nullptr;
   mp_status s = scratch_address(dev, &scratch);
   if (s != MP_OK) return s;
-  // Apart from the ticket head (zero-initialised with the array and left zero
-  // by every finished step), every byte a decode step reads was written
-  // earlier in the same step.
+  // Every byte of the array that a decode step reads was written earlier in
+  // the same step: the array needs no initialisation and no reset.
   return decode_impl(idx, Q, O, p, scratch, MP_STATIC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
-}
-
-extern "C" mp_status mp_decode_static_reset(void* stream) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MP_ECUDA;
-  void* scratch = nullptr;
-  mp_status s = scratch_address(dev, &scratch);
-  if (s != MP_OK) return s;
-  return cudaMemsetAsync(scratch, 0, kScratchTicketBytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MP_OK
-                                                                                                        : MP_ECUDA;
 }

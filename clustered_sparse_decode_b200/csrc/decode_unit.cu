@@ -1,0 +1,1180 @@
+// Decode step for bf16 caches: one kernel in which each (batch, KV head) unit
+// is decoded by one CTA, or by a cluster of k CTAs when there are few units
+// (k = 2, 4 or 8 keeps the grid near one CTA per SM).  The same engine runs
+// the dense baseline (every key attended exactly).
+//
+// "Multipole Attention for Efficient Long Context Reasoning" (arXiv abstract;
+// atlas.scime summary, "Approach"): the query scores every key centroid, the
+// best clusters up to a token budget are attended exactly, and every other
+// cluster enters the same softmax as one term with logit score + ln(size) and
+// its value centroid.
+//
+// Per unit, in one CTA (or cluster), every load of the cache by TMA:
+//   1. key centroids    128-row tiles of Kc: scores S[c][g] = scale q_g.Kc_c
+//                       (to the scratch, each read back by the thread that
+//                       wrote it or after a block barrier) and group scores
+//                       max_g S[c][g] (shared memory).
+//   2. selection        token-budgeted over the group scores max_g S[c][g]
+//                       (a cluster first gathers its CTAs' scores over
+//                       distributed shared memory): clusters in descending
+//                       score, ties to the lower slot, the crossing cluster
+//                       whole.  Meanwhile the producer already streams 3.:
+//                       its loads do not depend on the selection.
+//   3. value centroids  128-row tiles of Vc: the centroid terms of the
+//                       UNSELECTED non-empty clusters (logit S + ln n_c, value
+//                       Vc_c) enter the online softmax; selected clusters are
+//                       masked, so no term is ever added and taken out again.
+//   4. exact rows       the selected clusters' runs of the cluster-ordered
+//                       store, then the un-clustered tail, as 8-row boxes of
+//                       keys and values (one TMA each).  A run's last partial
+//                       box is placed to end at the run's end, overlapping the
+//                       run's previous box, and is issued one ring later, when
+//                       the overlapping rows are already in L2: DRAM reads each
+//                       row of the run once.
+//   5. combine          the eight warps' softmax states (and, in a cluster,
+//                       the CTAs' states over distributed shared memory)
+//                       merge into O.
+//
+// Warps: 8 compute warps in two groups of 4; group w computes the chunks
+// k = w (mod 2) of a ring of 32 KB chunks (d = 128), on mma.sync (bf16 in, fp32
+// accumulate); one producer warp fills the ring.  Every wait on the device is
+// bounded (then an error bit is set and the kernel winds down).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "stream_common.cuh"
+
+namespace mp {
+namespace unit {
+using namespace sc;
+
+constexpr int kCW = 8;                         // compute warps (two groups of 4)
+constexpr int kCT = kCW * kWarp;               // compute threads
+constexpr int kGW = 4;                         // warps per compute group
+constexpr int kThreads = kCT + kWarp;          // + one producer warp
+constexpr int kRows = 128;                     // centroid rows per chunk (keys or values only)
+constexpr int kDRows = 64;                     // dense chunks: key and value rows
+constexpr int kBoxes = 8;                      // 8-row boxes (keys and values) per exact chunk
+constexpr int kMaxNS = 12;                     // ring slots at most
+constexpr int kMinNS = 4;
+constexpr int kMaxSpt = 16;                    // selection: slots per compute thread
+constexpr int kMaxSlots = kMaxSpt * kCT;       // 4096
+constexpr int kMaxCluster = 8;
+constexpr int kSegCap = 64;                    // producer run queue: segments ...
+constexpr int kTailCap = 256;                  // ... and tail boxes waiting for their release
+constexpr int kSmemLimit = 232448;             // dynamic shared memory of one CTA per SM
+constexpr int kBarC = 2;                       // named barrier: compute threads
+
+enum Mode : int { M_FLAT = 0, M_DENSE = 1 };
+enum ChunkKind : int { K_KC = 0, K_VC = 1, K_BOX = 2, K_DENSE = 3, K_END = 4 };
+
+struct Args {
+  CUtensorMap tmA;             // M_FLAT: Kc, M_DENSE: K, as [units*rows][D] bf16, 64-column tiles (128-byte swizzle)
+  CUtensorMap tmB;             // M_FLAT: Vc, M_DENSE: V
+  CUtensorMap tmKV;            // M_FLAT: Kp and Vp as one map (columns, rows, [half,] key/value): 8-row boxes
+  const __nv_bfloat16* Q;      // [units][G][D]
+  __nv_bfloat16* O;            // [units][G][D]
+  const int32_t* off;          // M_FLAT: [units][slots + 1]
+  float* S;                    // M_FLAT: scratch [units][slots][SG] per-head scores (natural-log units)
+  uint8_t* sel_mask_out;       // optional [units][slots]
+  float* scores_out;           // optional [units][slots]
+  int32_t* err;
+  int units, k;                // k: CTAs per unit (cluster size)
+  int rows, rows_active;       // per unit: rows of the tile maps (slots | max_tokens) and rows to stream
+  int max_tokens, n_clustered, n_tail;
+  float scale;                 // score scale, natural-log units
+  int budget, approx;
+  long long timeout_ns;
+  // shared-memory plan (byte offsets from the 1024-aligned base)
+  int ns, o_meta, o_shat, o_offs, o_selm, o_wpre, o_q, o_red, o_bar, smem_bytes;
+};
+
+// What the producer tells the compute warps about the chunk in a ring slot.
+struct Meta {
+  int kind, cnt, p0, pad;      // cnt: rows (K_KC, K_VC, K_DENSE) or boxes (K_BOX); p0: first row
+  uint8_t lo[kBoxes], hi[kBoxes];   // K_BOX: valid rows [lo, hi) of each box
+  int row[kBoxes];             // K_BOX: first store row of each box (tensor-map row coordinate)
+};
+constexpr int kMetaBytes = 64;
+static_assert(sizeof(Meta) <= kMetaBytes, "meta");
+
+// A ring slot holds kRows centroid rows, kBoxes exact 8-row boxes (keys and
+// values) or kDRows dense rows (keys and values): 256 D bytes.
+template <int D>
+struct Geo {
+  static constexpr int SLOT = kRows * D * 2;
+  static constexpr int BOXB = 32 * D;              // one 8-row box: key rows, then value rows
+  static constexpr int DAREA = kDRows * D * 2;     // dense chunk: key rows, then value rows
+  static_assert(kBoxes * BOXB == SLOT && 2 * DAREA == SLOT, "chunk kinds share the slot size");
+};
+
+__host__ __device__ inline int r16(int x) { return (x + 15) & ~15; }
+__host__ __device__ inline int sg_of(int G) { return (G + 3) / 4 * 4; }
+
+// Shared-memory plan: the ring takes what the unit's tables leave (host and device).
+template <int D>
+__host__ __device__ inline void plan(Args& a, int mode, int slots, int G) {
+  const int sc = mode == M_FLAT ? (slots + 31) & ~31 : 0;
+  int o = 0;
+  const int meta = r16(kMaxNS * kMetaBytes);
+  const int shat = sc * 4;
+  const int offs = mode == M_FLAT ? r16((sc + 1) * 4) : 0;
+  const int selm = mode == M_FLAT ? r16(sc / 8) : 0;
+  const int wpre = mode == M_FLAT ? r16((sc / 32 + 1) * 4) : 0;
+  const int q = mode == M_FLAT ? kSegCap * 8 + kTailCap * 16 : 0;
+  const int red = mode == M_FLAT ? 1024 * 4 : 0;
+  const int bar = 2 * kMaxNS * 8 + 16;
+  const int fixed = meta + shat + offs + selm + wpre + q + red + bar;
+  // An even number of slots: chunk k goes to slot k % ns and to compute group
+  // k % 2, so every slot always serves the same group, which waits for that
+  // slot's phases one after the other (a wait never runs two phases ahead of
+  // the slot, where a parity test could not tell the phases apart).
+  int ns = (kSmemLimit - 1024 - fixed) / Geo<D>::SLOT;
+  ns = ns > kMaxNS ? kMaxNS : ns;
+  ns &= ~1;
+  a.ns = ns;
+  o = ns * Geo<D>::SLOT;
+  a.o_meta = o; o += meta;
+  a.o_shat = o; o += shat;
+  a.o_offs = o; o += offs;
+  a.o_selm = o; o += selm;
+  a.o_wpre = o; o += wpre;
+  a.o_q = o; o += q;
+  a.o_red = o; o += red;
+  a.o_bar = o; o += bar;
+  a.smem_bytes = o + 1024;     // + alignment slack
+}
+
+// ---------------------------------------------------------------------------
+// Cluster helpers (distributed shared memory)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return (int)r;
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync() { cluster_arrive(); cluster_wait(); }
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, int cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(cta));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_peer_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync %0, %1;\n" ::"n"(kBarC), "n"(kCT) : "memory"); }
+
+// ---------------------------------------------------------------------------
+// Selection over the group scores (compute threads).  Token-budgeted:
+// clusters by group score descending, ties to the lower slot, the shortest
+// prefix whose token count reaches the budget (the crossing cluster whole);
+// budget <= 0 selects nothing, a budget at or above all clustered tokens
+// selects every non-empty cluster.  The threshold tau (the largest key with
+// W(key >= tau) >= budget, keys being the order-preserving uint32 images of
+// the group scores) is found first through 256 equal-width score bins (when at
+// most 32 clusters fall into the crossing bin one warp sorts them), else by a
+// radix descent over 256-bin histograms of the keys.  shat: [slots] group
+// scores; writes the bitmask selm (complete after the final barrier).
+// ---------------------------------------------------------------------------
+template <int G>
+__device__ void select_smem(const Args& a, const float* shat, const int32_t* offs, uint32_t* selm, int* red,
+                            int* hist, int u, bool write_out) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slots = a.rows_active;
+  // thread tid owns slots tid + k kCT: a warp reads 32 consecutive slots (no
+  // bank conflicts) and the selection of 32 consecutive slots is one ballot
+  uint32_t key[kMaxSpt];
+  int w[kMaxSpt];
+  int wsum = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int k = 0; k < kMaxSpt; ++k) {
+    const int c = tid + k * kCT;
+    const bool in = c < slots;
+    const int cnt = in ? offs[c + 1] - offs[c] : 0;
+    const float sh = cnt > 0 ? shat[c] : -INFINITY;
+    key[k] = cnt > 0 ? ordered_key(sh) : 0u;
+    w[k] = cnt > 0 ? cnt : 0;
+    wsum += w[k];
+    if (cnt > 0) { kmin = min(kmin, key[k]); kmax = max(kmax, key[k]); }
+  }
+  {
+    const int ws_ = __reduce_add_sync(kFull, wsum);
+    const uint32_t mn = __reduce_min_sync(kFull, kmin), mx = __reduce_max_sync(kFull, kmax);
+    if (lane == 0) { red[warp] = ws_; red[kCW + warp] = (int)mn; red[2 * kCW + warp] = (int)mx; }
+    cbar();
+    wsum = 0; kmin = 0xffffffffu; kmax = 0u;
+#pragma unroll
+    for (int i = 0; i < kCW; ++i) {
+      wsum += red[i];
+      kmin = min(kmin, (uint32_t)red[kCW + i]);
+      kmax = max(kmax, (uint32_t)red[2 * kCW + i]);
+    }
+    cbar();
+  }
+  const int W = wsum;
+  const int mode = (a.budget <= 0 || W == 0) ? 0 : (W <= a.budget ? 1 : 2);   // none | all | threshold
+  uint32_t tau = 0u;
+  int ntie = 0, above = 0;
+  bool resolved = false;
+  if (mode == 2) {
+    const float smin = key_score(kmin), smax = key_score(kmax);
+    const float span = smax - smin, inv = 256.f / span;
+    if (isfinite(smin) && isfinite(smax) && span > 0.f && isfinite(span) && isfinite(inv)) {
+      auto fbin = [&](uint32_t kk) { return min(255, (int)((key_score(kk) - smin) * inv)); };
+      int* lst = hist + 256;                                // [32][3] candidates of the crossing bin
+      for (int i = tid; i < 256; i += kCT) hist[i] = 0;
+      if (tid == 0) red[3] = 0;
+      cbar();
+#pragma unroll
+      for (int k = 0; k < kMaxSpt; ++k)
+        if (w[k] > 0) atomicAdd(hist + fbin(key[k]), w[k]);
+      cbar();
+      if (warp == 0) {
+        int bl[8], ls = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { bl[i] = hist[8 * lane + i]; ls += bl[i]; }
+        int suf = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(kFull, suf, o);
+          if (lane + o < 32) suf += y;
+        }
+        int run = suf - ls, found = -1, ab = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (found < 0 && run + bl[i] >= a.budget) { found = 8 * lane + i; ab = run; }
+          run += bl[i];
+        }
+        const unsigned m = __ballot_sync(kFull, found >= 0);
+        const int src = 31 - __clz(m);
+        const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
+        if (lane == 0) { red[0] = fb; red[1] = fa; }
+      }
+      cbar();
+      const int fb = red[0], ab = red[1];
+#pragma unroll
+      for (int k = 0; k < kMaxSpt; ++k)
+        if (w[k] > 0 && fbin(key[k]) == fb) {
+          const int pos = atomicAdd(red + 3, 1);
+          if (pos < 32) { lst[3 * pos] = (int)key[k]; lst[3 * pos + 1] = tid + k * kCT; lst[3 * pos + 2] = w[k]; }
+        }
+      cbar();
+      const int nc = red[3];
+      if (nc <= 32) {
+        if (warp == 0) {
+          // lane l holds candidate l; empty lanes sort last with weight 0
+          uint64_t v = lane < nc ? ((uint64_t)(uint32_t)lst[3 * lane] << 32) | (uint32_t)(0xffffffffu - (uint32_t)lst[3 * lane + 1])
+                                 : 0ull;
+          int wl = lane < nc ? lst[3 * lane + 2] : 0;
+#pragma unroll
+          for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+              const uint64_t ov = __shfl_xor_sync(kFull, v, jj);
+              const int ow = __shfl_xor_sync(kFull, wl, jj);
+              const bool up = ((lane & kk) == 0) == ((lane & jj) == 0);   // this lane keeps the larger
+              if (up ? ov > v : ov < v) { v = ov; wl = ow; }
+            }
+          }
+          int inc = wl;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += y;
+          }
+          const unsigned cross = __ballot_sync(kFull, lane < nc && ab + inc >= a.budget);
+          const uint32_t t = (uint32_t)(__shfl_sync(kFull, v, __ffs(cross) - 1) >> 32);
+          const uint32_t kl = (uint32_t)(v >> 32);
+          const int gt = __reduce_add_sync(kFull, lane < nc && kl > t ? wl : 0);
+          const int nt = __popc(__ballot_sync(kFull, lane < nc && kl == t));
+          if (lane == 0) { red[0] = (int)t; red[1] = ab + gt; red[2] = nt; }
+        }
+        cbar();
+        tau = (uint32_t)red[0];
+        above = red[1];
+        ntie = red[2];
+        resolved = true;
+      }
+      cbar();
+    }
+  }
+  if (mode == 2 && !resolved) {
+    uint32_t lo = kmin;
+    int nb = kmax == kmin ? 0 : 32 - __clz(kmax - kmin);
+    above = 0;
+    int* hcnt = hist + 256;
+    ntie = -1;
+    while (nb > 0) {
+      const int sh = max(nb - 8, 0);
+      for (int i = tid; i < 256; i += kCT) { hist[i] = 0; hcnt[i] = 0; }
+      cbar();
+      const unsigned long long hi_excl = (unsigned long long)lo + (1ull << nb);
+#pragma unroll
+      for (int k = 0; k < kMaxSpt; ++k)
+        if (w[k] > 0 && key[k] >= lo && (unsigned long long)key[k] < hi_excl) {
+          const int bin = (int)((key[k] - lo) >> sh);
+          atomicAdd(hist + bin, w[k]);
+          if (sh == 0) atomicAdd(hcnt + bin, 1);
+        }
+      cbar();
+      if (warp == 0) {
+        int bl[8], ls = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { bl[i] = hist[8 * lane + i]; ls += bl[i]; }
+        int suf = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(kFull, suf, o);
+          if (lane + o < 32) suf += y;
+        }
+        int run = above + suf - ls;
+        int found = -1, ab = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (found < 0 && run + bl[i] >= a.budget) { found = 8 * lane + i; ab = run; }
+          run += bl[i];
+        }
+        const unsigned m = __ballot_sync(kFull, found >= 0);
+        const int src = 31 - __clz(m);
+        const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
+        if (lane == 0) { red[0] = fb; red[1] = fa; red[2] = hcnt[fb]; }
+      }
+      cbar();
+      const int b = red[0];
+      above = red[1];
+      if (sh == 0) ntie = red[2];
+      lo += (uint32_t)b << sh;
+      nb = sh;
+      cbar();
+    }
+    tau = lo;
+  }
+  const int need = mode == 2 ? a.budget - above : 0;   // tokens still to take among the ties at tau
+  // several clusters exactly at tau: they are taken in slot order, slot tid + k kCT
+  // after every slot of rows k' < k and of lower threads in row k
+  int tie_before[kMaxSpt];
+#pragma unroll
+  for (int k = 0; k < kMaxSpt; ++k) tie_before[k] = 0;
+  if (mode == 2 && ntie != 1) {
+    int row_base = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxSpt; ++k) {
+      const int tw = (key[k] == tau && w[k] > 0) ? w[k] : 0;
+      int inc = tw;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += y;
+      }
+      if (lane == 31) red[64 + warp] = inc;
+      cbar();
+      int pre = 0, row = 0;
+#pragma unroll
+      for (int i = 0; i < kCW; ++i) {
+        pre += i < warp ? red[64 + i] : 0;
+        row += red[64 + i];
+      }
+      tie_before[k] = row_base + pre + inc - tw;
+      row_base += row;
+      cbar();
+    }
+  }
+  // the selection of slots [32 (8 k + warp), + 32): one ballot, one word
+#pragma unroll
+  for (int k = 0; k < kMaxSpt; ++k) {
+    bool sel = false;
+    if (w[k] > 0) {
+      if (mode == 1) sel = true;
+      else if (mode == 2) sel = key[k] > tau || (key[k] == tau && tie_before[k] < need);
+    }
+    const unsigned bits = __ballot_sync(kFull, sel);
+    if (lane == 0 && k * kCT + warp * 32 < slots) selm[k * kCW + warp] = bits;
+    if (write_out) {
+      const int c = tid + k * kCT;
+      if (c < slots) {
+        if (a.sel_mask_out) a.sel_mask_out[(size_t)u * a.rows + c] = sel ? 1 : 0;
+        if (a.scores_out) a.scores_out[(size_t)u * a.rows + c] = w[k] > 0 ? key_score(key[k]) : -INFINITY;
+      }
+    }
+  }
+  if (write_out) {
+    // slots of blocks that hold no tokens yet
+    for (int c = slots + tid; c < a.rows; c += kCT) {
+      if (a.sel_mask_out) a.sel_mask_out[(size_t)u * a.rows + c] = 0;
+      if (a.scores_out) a.scores_out[(size_t)u * a.rows + c] = -INFINITY;
+    }
+  }
+  cbar();
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+template <int D, int G, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant__ Args a) {
+  using Gm = Geo<D>;
+  constexpr int SG = (G + 3) / 4 * 4;      // floats per score row (16-byte multiple)
+  constexpr int CR = MODE == M_FLAT ? kRows : kDRows;   // rows per chunk of the first stream
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  float* shat = reinterpret_cast<float*>(smem + a.o_shat);            // [rows] group scores max_g S
+  int32_t* offs = reinterpret_cast<int32_t*>(smem + a.o_offs);        // [rows + 1] run offsets
+  uint32_t* selm = reinterpret_cast<uint32_t*>(smem + a.o_selm);      // selection bitmask
+  int32_t* wpre = reinterpret_cast<int32_t*>(smem + a.o_wpre);        // selected clusters before each word
+  int* red = reinterpret_cast<int*>(smem + a.o_red);
+  const uint32_t full0 = sb + a.o_bar, empty0 = full0 + kMaxNS * 8, selready = empty0 + kMaxNS * 8;
+  auto meta = [&](int slot) { return reinterpret_cast<Meta*>(smem + a.o_meta + slot * kMetaBytes); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = a.k;
+  const int rank = K > 1 ? cluster_rank() : 0;
+  const int u = blockIdx.x / K;
+  const int NS = a.ns;
+  const long long deadline = gtimer() + a.timeout_ns;
+  // this CTA's chunks [c_lo, c_hi) of the unit's first stream
+  const int nch = (a.rows_active + CR - 1) / CR;
+  const int c_lo = (int)((long long)rank * nch / K), c_hi = (int)((long long)(rank + 1) * nch / K);
+  const int n1 = c_hi - c_lo;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(full0 + 8 * i, 1);           // the producer's arrival (+ the TMA bytes it announces)
+      mbar_init(empty0 + 8 * i, kGW);        // one arrival per warp of the chunk's compute group
+    }
+    mbar_init(selready, 1);                  // the selection is in shared memory
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (MODE == M_FLAT && warp < kCW) {
+    // the unit's run offsets (counts of every slot), for the centroid terms and the selection
+    const int32_t* ou = a.off + (size_t)u * (a.rows + 1);
+    for (int i = threadIdx.x; i <= a.rows_active; i += kCT) offs[i] = __ldg(ou + i);
+  }
+  __syncthreads();
+
+  if (warp == kCW) {
+    // ============================ producer ============================
+    int k = 0;              // chunk counter (all streams)
+    bool ok = true;
+    auto acquire = [&](int kk) -> bool {   // wait until the slot of chunk kk is free
+      const int slot = kk % NS;
+      bool got = true;
+      if (kk >= NS && lane == 0) got = mbar_wait(empty0 + 8 * slot, ((kk / NS) - 1) & 1, deadline);
+      got = __shfl_sync(kFull, got ? 1 : 0, 0) != 0;
+      if (!got && lane == 0) set_error(a.err, E_TIMEOUT);
+      return got;
+    };
+    // ---- first stream: key centroid tiles (flat) or key and value tiles (dense) ----
+    for (int x = c_lo; x < c_hi && ok; ++x, ++k) {
+      if (!(ok = acquire(k))) break;
+      const int slot = k % NS;
+      if (lane == 0) {
+        Meta* m = meta(slot);
+        const int p0 = x * CR;
+        m->kind = MODE == M_FLAT ? K_KC : K_DENSE;
+        m->cnt = min(CR, a.rows_active - p0);
+        m->p0 = p0;
+        const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
+        const int y = u * a.rows + p0;
+        mbar_arrive_tx(bar, (uint32_t)Gm::SLOT);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) tma_2d(dst + h * (CR * 128), &a.tmA, 64 * h, y, bar);
+        if (MODE == M_DENSE) {
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) tma_2d(dst + Gm::DAREA + h * (CR * 128), &a.tmB, 64 * h, y, bar);
+        }
+      }
+    }
+    if constexpr (MODE == M_FLAT) {
+      if (K > 1) cluster_arrive();         // (1): nothing of this warp's is read by the peers
+      // ---- value centroid tiles: their loads do not wait for the selection ----
+      if (a.approx) {
+        for (int x = c_lo; x < c_hi && ok; ++x, ++k) {
+          if (!(ok = acquire(k))) break;
+          const int slot = k % NS;
+          if (lane == 0) {
+            Meta* m = meta(slot);
+            const int p0 = x * kRows;
+            m->kind = K_VC;
+            m->cnt = min(kRows, a.rows_active - p0);
+            m->p0 = p0;
+            const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
+            mbar_arrive_tx(bar, (uint32_t)Gm::SLOT);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) tma_2d(dst + h * (kRows * 128), &a.tmB, 64 * h, u * a.rows + p0, bar);
+          }
+        }
+      }
+      // ---- exact rows: needs the selection ----
+      bool got = true;
+      if (lane == 0) got = mbar_wait(selready, 0, deadline);
+      if (!__shfl_sync(kFull, got ? 1 : 0, 0)) {
+        if (lane == 0) set_error(a.err, E_TIMEOUT);
+        ok = false;
+      }
+      const int nw = (a.rows_active + 31) >> 5;
+      int tot = 0;
+      for (int w0 = 0; w0 < nw; w0 += 32) {   // per-word prefix of selected-cluster counts
+        const int wi = w0 + lane;
+        const int c = wi < nw ? __popc(selm[wi]) : 0;
+        int inc = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, inc, o);
+          if (lane >= o) inc += y;
+        }
+        if (wi < nw) wpre[wi] = tot + inc - c;
+        tot += __shfl_sync(kFull, inc, 31);
+      }
+      if (lane == 0) wpre[nw] = tot;
+      __syncwarp();
+      // this CTA's share: selected clusters of rank [r_lo, r_hi), tail rows [t_lo, t_hi)
+      const int nsel = tot;
+      const int r_lo = (int)((long long)rank * nsel / K), r_hi = (int)((long long)(rank + 1) * nsel / K);
+      const int t_lo = a.n_clustered + (int)((long long)rank * a.n_tail / K);
+      const int t_hi = a.n_clustered + (int)((long long)(rank + 1) * a.n_tail / K);
+      const int unit_row = u * a.max_tokens;
+      const int zero_row = a.units * a.max_tokens;   // a box wholly past the stores: zero-filled, no reads
+      const int DM = kBoxes * NS;                    // a tail box waits this many main boxes: one ring
+      // Run queue: segments {first row, full boxes (> 0) | -(rows of a run under 8 rows)}
+      // and tail boxes {first row, first valid row, release (main boxes issued), 0}.
+      int2* segq = reinterpret_cast<int2*>(smem + a.o_q);
+      int4* tailq = reinterpret_cast<int4*>(smem + a.o_q + kSegCap * 8);
+      int sh = 0, stl = 0, th = 0, ttl = 0;          // ring heads and tails (monotone, warp-uniform)
+      int rk = r_lo, seg_off = 0;                    // next rank to enqueue; boxes of the head segment issued
+      bool tail_run = t_lo < t_hi;                   // the un-clustered tail still to enqueue
+      long long mb_enq = 0, mb_iss = 0;              // main boxes enqueued / issued
+      // enqueue one run per lane (valid lanes): its full boxes as a segment, its
+      // last < 8 rows as a tail box ending at the run's end, released one ring later
+      auto enqueue = [&](bool valid, int st, int cnt) {
+        const int nf = cnt >> 3, rem = cnt & 7;
+        const unsigned vm = __ballot_sync(kFull, valid);
+        const unsigned lt = (1u << lane) - 1u;
+        if (valid) segq[(stl + __popc(vm & lt)) % kSegCap] = make_int2(st, nf > 0 ? nf : -cnt);
+        int mb = valid ? (nf > 0 ? nf : 1) : 0, inc = mb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const bool tl = valid && nf > 0 && rem > 0;
+        const unsigned tm = __ballot_sync(kFull, tl);
+        if (tl)
+          tailq[(ttl + __popc(tm & lt)) % kTailCap] =
+              make_int4(st + cnt - 8, 8 - rem, (int)(mb_enq + inc + DM), 0);
+        stl += __popc(vm);
+        ttl += __popc(tm);
+        mb_enq += __shfl_sync(kFull, inc, 31);
+      };
+      // the next up to 32 selected clusters, one per lane, located by rank
+      auto refill = [&]() {
+        if (rk < r_hi) {
+          const int n = min(32, r_hi - rk);
+          bool valid = false;
+          int st = 0, cnt = 0;
+          if (lane < n) {
+            const int r = rk + lane;
+            int lo = 0, hi = nw - 1;                 // the word holding rank r: the last w with wpre[w] <= r
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (wpre[mid] <= r) lo = mid; else hi = mid - 1;
+            }
+            uint32_t word = selm[lo];
+            for (int i = wpre[lo]; i < r && word; ++i) word &= word - 1;
+            if (word == 0u) {
+              set_error(a.err, E_BAD_LIST);
+            } else {
+              const int sl = (lo << 5) + __ffs(word) - 1;
+              st = offs[sl];
+              cnt = offs[sl + 1] - st;
+              if (st < 0 || cnt < 1 || st + cnt > a.max_tokens) set_error(a.err, E_BAD_OFFSET);
+              else valid = true;
+            }
+          }
+          enqueue(valid, st, cnt);
+          rk += n;
+        } else if (tail_run) {
+          enqueue(lane == 0, t_lo, t_hi - t_lo);
+          tail_run = false;
+        }
+      };
+      for (;;) {
+        // keep at least one chunk of segments queued (while the tail-box ring has room)
+        while ((rk < r_hi || tail_run) && stl - sh < kBoxes && ttl - th <= kTailCap - 32) refill();
+        const bool done_enq = rk >= r_hi && !tail_run;
+        if (!ok || (sh == stl && th == ttl && done_enq)) break;
+        if (!(ok = acquire(k))) break;
+        const int slot = k % NS;
+        Meta* m = meta(slot);
+        // lane-parallel assembly: lane b < kBoxes works out box b of the chunk.
+        // First the tail boxes whose runs' full boxes were issued one ring ago
+        // (the rows they share with those boxes are in L2 by now), in release
+        // order; then main boxes from the next segments.
+        const unsigned lo8 = (1u << kBoxes) - 1u;
+        int4 tv = make_int4(0, 0, 0, 0);
+        const bool has_t = lane < kBoxes && th + lane < ttl;
+        if (has_t) tv = tailq[(th + lane) % kTailCap];
+        int nt = __ffs(~(__ballot_sync(kFull, has_t && tv.z <= mb_iss) & lo8)) - 1;   // released prefix
+        int2 sg = make_int2(0, 0);
+        int sb_cnt = 0;                          // boxes left in segment sh + lane
+        if (lane < kBoxes && sh + lane < stl) {
+          sg = segq[(sh + lane) % kSegCap];
+          sb_cnt = (sg.y > 0 ? sg.y : 1) - (lane == 0 ? seg_off : 0);
+        }
+        int incl = sb_cnt;
+#pragma unroll
+        for (int o = 1; o < kBoxes; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int avail = __shfl_sync(kFull, incl, kBoxes - 1);
+        int nm = min(kBoxes - nt, avail);        // main boxes in this chunk
+        if (nm == 0) {
+          // no main box left (or none queued): waiting tail boxes go now
+          nt = min(kBoxes, ttl - th);
+        } else if (sh + kBoxes >= stl && done_enq && nm == avail) {
+          // the last main boxes: released or not, tail boxes fill the chunk
+          nt = min(kBoxes - nm, ttl - th);
+        }
+        int row = 0, blo = 0, bhi = 0;
+        bool on = false;
+        if (lane < nt) {
+          row = unit_row + tv.x;
+          blo = tv.y;
+          bhi = 8;
+          on = true;
+        }
+        const int mi = lane - nt;                // main box number in this chunk
+        // segment of main box mi: the first lane j with incl_j > mi
+        int seg_j = 0;
+#pragma unroll
+        for (int jj = 0; jj < kBoxes; ++jj) seg_j += (__shfl_sync(kFull, incl, jj) <= mi) ? 1 : 0;
+        const int incl_prev = __shfl_sync(kFull, incl, max(seg_j - 1, 0));   // every lane takes part
+        const int before = seg_j > 0 ? incl_prev : 0;
+        const int2 sj = make_int2(__shfl_sync(kFull, sg.x, min(seg_j, kBoxes - 1)),
+                                  __shfl_sync(kFull, sg.y, min(seg_j, kBoxes - 1)));
+        if (lane < kBoxes && mi >= 0 && mi < nm) {
+          const int off_in = mi - before + (seg_j == 0 ? seg_off : 0);
+          if (sj.y > 0) { row = unit_row + sj.x + 8 * off_in; blo = 0; bhi = 8; }
+          else { row = unit_row + sj.x; blo = 0; bhi = -sj.y; }   // a run under 8 rows: the rows after it are masked
+          on = true;
+        }
+        int nb = nt + nm;
+        if ((nb & 1) && lane == nb) { row = zero_row; blo = 0; bhi = 0; on = true; }   // all-zero partner box
+        nb += nb & 1;
+        if (on) {
+          m->lo[lane] = (uint8_t)blo;
+          m->hi[lane] = (uint8_t)bhi;
+          m->row[lane] = row;
+        }
+        // advance the queues past this chunk's boxes
+        {
+          const int full_segs = __popc(__ballot_sync(kFull, lane < kBoxes && sb_cnt > 0 && incl <= nm) & lo8);
+          const int incl_last = __shfl_sync(kFull, incl, max(full_segs - 1, 0));   // every lane takes part
+          const int used = full_segs > 0 ? incl_last : 0;
+          seg_off = full_segs > 0 ? nm - used : seg_off + nm;
+          sh += full_segs;
+          th += nt;
+          mb_iss += nm;
+        }
+        if (lane == 0) {
+          m->kind = K_BOX;
+          m->cnt = nb;
+        }
+        __syncwarp();
+        const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
+        if (lane == 0) mbar_arrive_tx(bar, (uint32_t)(nb * Gm::BOXB));
+        __syncwarp();
+        if (lane < nb) tma_box<D>(dst + lane * Gm::BOXB, &a.tmKV, row, bar);
+        ++k;
+      }
+    }
+    // end markers: one for each compute group
+    for (int e = 0; e < 2 && ok; ++e, ++k) {
+      if (!(ok = acquire(k))) break;
+      const int slot = k % NS;
+      if (lane == 0) {
+        meta(slot)->kind = K_END;
+        meta(slot)->cnt = 0;
+        mbar_arrive(full0 + 8 * slot);
+      }
+      __syncwarp();
+    }
+    if (K > 1) {
+      if (MODE == M_FLAT) cluster_wait();  // (1)
+      cluster_sync();                      // (2) the CTA partials are complete
+      cluster_sync();                      // (3) every CTA has read its peers' partials
+    }
+    return;
+  }
+
+  // ============================ compute warps ============================
+  const int grp = warp / kGW, wg = warp % kGW;
+  const float qk2 = a.scale * kLog2e;
+  WarpSoftmax<D, G> ws;
+  ws.reset();
+  ws.load_q(a.Q + (size_t)u * G * D, lane);
+  bool alive = true;
+  auto wait_full = [&](int k) -> bool {
+    if (mbar_wait(full0 + 8 * (k % NS), (k / NS) & 1, deadline)) return true;
+    if (lane == 0) set_error(a.err, E_TIMEOUT);
+    alive = false;
+    return false;
+  };
+  // ---- first stream (this group's chunks k = grp, grp + 2, ...) ----
+  for (int k = grp; k < n1 && alive; k += 2) {
+    if (!wait_full(k)) break;
+    const int slot = k % NS;
+    const Meta* m = meta(slot);
+    const int cnt = m->cnt, p0 = m->p0;
+    const uint32_t dst = sb + slot * Gm::SLOT;
+    if constexpr (MODE == M_FLAT) {
+      // key centroids: 32 rows per warp, scores into shared memory
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r16 = wg * 32 + t * 16;
+        if (r16 < cnt) {
+          float z[2][2];
+          ws.template qk<false, kRows>(dst, r16, lane, z);
+          const bool wr = !WarpSoftmax<D, G>::lo_cols(lane);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
+            float gmax = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int h = WarpSoftmax<D, G>::col_head(lane, j);
+              const float sc = z[i][j] * a.scale;
+              if (wr && h >= 0) {
+                gmax = fmaxf(gmax, sc);
+                if (r < cnt) a.S[((size_t)u * a.rows + p0 + r) * SG + h] = sc;
+              }
+            }
+            // the group score of the row: max over the four lanes holding its columns
+            gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 1));
+            gmax = fmaxf(gmax, __shfl_xor_sync(kFull, gmax, 2));
+            if ((lane & 3) == 0 && r < cnt) shat[p0 + r] = gmax;
+          }
+        }
+      }
+    } else {
+      // dense: 16 key and value rows per warp, every key exact
+      const int r16 = wg * 16;
+      if (r16 < cnt) {
+        float z[2][2];
+        ws.template qk<false, kDRows>(dst, r16, lane, z);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            z[i][j] = (WarpSoftmax<D, G>::col_head(lane, j) >= 0 && r < cnt) ? z[i][j] * qk2 : -INFINITY;
+        }
+        ws.template update<false, kDRows>(dst + Gm::DAREA, r16, lane, z, 1.f);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+  }
+  if constexpr (MODE == M_FLAT) {
+    // ---- selection ----
+    cbar();                                // this CTA's scores are in shared memory
+    if (K > 1) {
+      cluster_arrive();                    // (1) ... and every peer's
+      cluster_wait();
+      // the peers' group scores: slots [c_lo', c_hi') * kRows of CTA r'
+      for (int r = 0; r < K; ++r) {
+        if (r == rank) continue;
+        const int lo = (int)((long long)r * nch / K) * kRows;
+        const int hi = min(a.rows_active, (int)((long long)(r + 1) * nch / K) * kRows);
+        const uint32_t base = peer_addr(smem_u32(shat), r);
+        for (int i = lo + (int)threadIdx.x; i < hi; i += kCT) shat[i] = __uint_as_float(ld_peer_u32(base + 4u * i));
+      }
+      cbar();
+    }
+    select_smem<G>(a, shat, offs, selm, red, red + 256, u, rank == 0);
+    if (threadIdx.x == 0) mbar_arrive(selready);   // the producer may walk the selection
+  }
+  // ---- value centroids and exact rows ----
+  for (int k = n1 + ((grp - n1) % 2 + 2) % 2; alive; k += 2) {
+    // a value-centroid chunk: its scores come from the scratch (written by the
+    // key stream before the selection's barriers); load them before the wait
+    float sv[2][2][2];
+    const bool vc_chunk = MODE == M_FLAT && a.approx && k < 2 * n1;
+    if (vc_chunk) {
+      const int p0 = (c_lo + k - n1) * kRows;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = p0 + wg * 32 + t * 16 + WarpSoftmax<D, G>::zrow(lane, i);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int h = WarpSoftmax<D, G>::col_head(lane, j);
+            sv[t][i][j] = (h >= 0 && r < a.rows_active) ? __ldcg(a.S + ((size_t)u * a.rows + r) * SG + h) : 0.f;
+          }
+        }
+    }
+    if (!wait_full(k)) break;
+    const int slot = k % NS;
+    const Meta* m = meta(slot);
+    const int kind = m->kind, cnt = m->cnt;
+    if (kind == K_END) break;
+    const uint32_t base = sb + slot * Gm::SLOT;
+    if (kind == K_VC) {
+      // value centroids of the unselected non-empty clusters: logit S + ln n
+      const int p0 = m->p0;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int r16 = wg * 32 + t * 16;
+        if (r16 < cnt) {
+          float z[2][2];
+          bool any = false;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
+            const int s = p0 + r;
+            const int n = r < cnt ? offs[s + 1] - offs[s] : 0;
+            const bool take = n > 0 && !((selm[s >> 5] >> (s & 31)) & 1u);
+            const float lg = log2f((float)n);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int h = WarpSoftmax<D, G>::col_head(lane, j);
+              z[i][j] = (take && h >= 0) ? sv[t][i][j] * kLog2e + lg : -INFINITY;
+              any |= take && h >= 0;
+            }
+          }
+          if (__any_sync(kFull, any)) ws.template update<false, kRows>(base, r16, lane, z, 1.f);
+        }
+      }
+    } else if (kind == K_BOX) {
+      const int r16 = wg * 16;
+      if (2 * wg < cnt) {
+        float z[2][2];
+        ws.template qk<true, kRows>(base, r16, lane, z);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int bx = 2 * wg + i;            // rows 8 i .. 8 i + 7 of this warp's tile are box bx
+          const int blo = m->lo[bx], bhi = m->hi[bx];
+          const int rb = lane >> 2;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            z[i][j] = (WarpSoftmax<D, G>::col_head(lane, j) >= 0 && rb >= blo && rb < bhi) ? z[i][j] * qk2 : -INFINITY;
+        }
+        ws.template update<true, kRows>(base + Gm::BOXB / 2, r16, lane, z, 1.f);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+  }
+  // ---- combine ----
+  cbar();                                  // every chunk is consumed: the ring is free
+  float* pm = reinterpret_cast<float*>(smem);                 // [kCW][G]
+  float* pl = pm + kCW * G;                                   // [kCW][G]
+  float* pacc = pl + kCW * G;                                 // [kCW][G][D]
+  float* cpart = pacc + kCW * G * D;                          // CTA partial: m[SG], l[SG], acc[G][D]
+  ws.store(pm + warp * G, pl + warp * G, pacc + (size_t)warp * G * D, lane);
+  cbar();
+  constexpr int NE = G * D / 4;            // float4 groups of the output rows
+  for (int e = threadIdx.x; e < NE; e += kCT) {
+    const int g = (e * 4) / D, d = (e * 4) % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < kCW; ++p) M = fmaxf(M, pm[p * G + g]);
+    float L = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int p = 0; p < kCW; ++p) {
+        const float mp_ = pm[p * G + g];
+        const float f = mp_ == -INFINITY ? 0.f : ex2(mp_ - M);
+        const float4 x = *reinterpret_cast<const float4*>(pacc + ((size_t)p * G + g) * D + d);
+        o.x += f * x.x; o.y += f * x.y; o.z += f * x.z; o.w += f * x.w;
+        L += f * pl[p * G + g];
+      }
+    }
+    if (K == 1) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat16* out = a.O + ((size_t)u * G + g) * D + d;
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16(o.x * inv, o.y * inv), pack_bf16(o.z * inv, o.w * inv));
+    } else {
+      if (d == 0) { cpart[g] = M; cpart[SG + g] = L; }
+      *reinterpret_cast<float4*>(cpart + 2 * SG + g * D + d) = o;
+    }
+  }
+  if (K > 1) {
+    cbar();
+    cluster_sync();                        // (2) every CTA's partial is complete
+    // this CTA writes the float4 groups [e_lo, e_hi) of the unit's output
+    const int e_lo = rank * NE / K, e_hi = (rank + 1) * NE / K;
+    const uint32_t cp_local = smem_u32(cpart);
+    for (int e = e_lo + (int)threadIdx.x; e < e_hi; e += kCT) {
+      const int g = (e * 4) / D, d = (e * 4) % D;
+      float M = -INFINITY;
+      for (int r = 0; r < K; ++r) M = fmaxf(M, __uint_as_float(ld_peer_u32(peer_addr(cp_local, r) + 4u * g)));
+      float L = 0.f;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+        for (int r = 0; r < K; ++r) {
+          const uint32_t pb = peer_addr(cp_local, r);
+          const float mr = __uint_as_float(ld_peer_u32(pb + 4u * g));
+          if (mr == -INFINITY) continue;
+          const float f = ex2(mr - M);
+          const float lr = __uint_as_float(ld_peer_u32(pb + 4u * (SG + g)));
+          const float4 x = ld_peer_f4(pb + 4u * (2 * SG + g * D + d));
+          o.x += f * x.x; o.y += f * x.y; o.z += f * x.z; o.w += f * x.w;
+          L += f * lr;
+        }
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat16* out = a.O + ((size_t)u * G + g) * D + d;
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16(o.x * inv, o.y * inv), pack_bf16(o.z * inv, o.w * inv));
+    }
+    cluster_sync();                        // (3) peers are done reading this CTA's partial
+  }
+}
+
+}  // namespace unit
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+// Scratch of the unit kernel: the per-head scores [units][slots][SG] fp32
+// (group scores, selection and partial states stay in shared memory).
+size_t unit_scratch_bytes(const mp_config& c, int slots) {
+  const size_t U = (size_t)c.batch * c.kv_heads;
+  const int G = c.q_heads / c.kv_heads;
+  return (U * slots * unit::sg_of(G) * 4 + 255) & ~(size_t)255;
+}
+
+static int unit_ring_slots(int D, int G, int mode, int slots) {
+  unit::Args a{};
+  if (D == 128) unit::plan<128>(a, mode, slots, G);
+  else unit::plan<64>(a, mode, slots, G);
+  return a.ns;
+}
+
+// The index shapes the unit kernel takes: flat bf16, d 64 or 128, G in {1, 2,
+// 4, 8}, at most 4096 slots whose scores leave room for a ring of at least 4
+// chunks in shared memory, store rows addressable by the tensor maps.
+bool unit_supported(const mp_config& c, int slots) {
+  const int G = c.q_heads / c.kv_heads;
+  const int64_t U = (int64_t)c.batch * c.kv_heads;
+  return c.levels == 1 && c.dtype == MP_BF16 && (c.head_dim == 64 || c.head_dim == 128) &&
+         (G == 1 || G == 2 || G == 4 || G == 8) && slots <= unit::kMaxSlots &&
+         U * c.max_tokens + 8 < (int64_t)INT32_MAX && U * slots < (int64_t)INT32_MAX &&
+         U * unit::kMaxCluster < (int64_t)INT32_MAX &&
+         unit_ring_slots(c.head_dim, G, unit::M_FLAT, slots) >= unit::kMinNS;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 unit_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// rows x D bf16 matrix, tiles of 64 columns x box_rows rows, 128-byte swizzle
+static bool encode_tiles(CUtensorMap* tm, const void* base, uint64_t rows, int D, int box_rows) {
+  auto fn = unit_encoder();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Kp and Vp ([rows][D] bf16 each, Vp after Kp) as one map whose outermost
+// dimension steps from Kp to Vp: an 8-row box lands as [key/value][64-column
+// half][8 rows][128 bytes], 128-byte swizzle.  The map covers exactly the two
+// stores; box rows past them read as zeros.
+static bool encode_boxes(CUtensorMap* tm, const void* Kp, const void* Vp, uint64_t rows, int D) {
+  auto fn = unit_encoder();
+  if (!fn) return false;
+  const intptr_t kv = reinterpret_cast<const char*>(Vp) - reinterpret_cast<const char*>(Kp);
+  if (kv < (intptr_t)(rows * D * 2) || (kv & 15) != 0 || kv >= ((intptr_t)1 << 40)) return false;
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (D == 128) {
+    cuuint64_t gdim[4] = {64, rows, 2, 2};
+    cuuint64_t gstride[3] = {256, 128, (cuuint64_t)kv};
+    cuuint32_t box[4] = {64, 8, 2, 2};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(Kp), gdim, gstride, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  cuuint64_t gdim[3] = {64, rows, 2};
+  cuuint64_t gstride[2] = {128, (cuuint64_t)kv};
+  cuuint32_t box[3] = {64, 8, 2};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(Kp), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int G, int MODE>
+static cudaError_t launch_unit_t(unit::Args& a, cudaStream_t st) {
+  auto kern = unit::unit_decode<D, G, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(a.units * a.k));
+  cfg.blockDim = dim3(unit::kThreads);
+  cfg.dynamicSmemBytes = a.smem_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.k;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.k > 1 ? 1 : 0;
+  if (a.k > 1) {
+    // the cluster must fit on the device with this kernel's shared memory
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1) {
+      cudaGetLastError();
+      a.k = 1;
+      cfg.gridDim = dim3((unsigned)a.units);
+      cfg.numAttrs = 0;
+    }
+  }
+  return cudaLaunchKernelEx(&cfg, kern, (const unit::Args)a);
+}
+
+template <int D, int MODE>
+static cudaError_t launch_unit_d(int G, unit::Args& a, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_unit_t<D, 1, MODE>(a, st);
+    case 2: return launch_unit_t<D, 2, MODE>(a, st);
+    case 4: return launch_unit_t<D, 4, MODE>(a, st);
+    case 8: return launch_unit_t<D, 8, MODE>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int MODE>
+static cudaError_t launch_unit(int D, int G, unit::Args& a, cudaStream_t st) {
+  if (D == 128) {
+    unit::plan<128>(a, MODE, a.rows, G);
+    return launch_unit_d<128, MODE>(G, a, st);
+  }
+  unit::plan<64>(a, MODE, a.rows, G);
+  return launch_unit_d<64, MODE>(G, a, st);
+}
+
+// CTAs per unit: clusters of k CTAs cover the SMs, each CTA with at least two
+// chunks of the first stream; the caller's split count (n_split > 0) overrides it
+static int cluster_size(int64_t units, int chunks, int n_split) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int k = 1;
+  if (n_split > 0) {
+    while (k * 2 <= std::min(n_split, unit::kMaxCluster)) k *= 2;
+  } else {
+    while (k * 2 <= unit::kMaxCluster && units * k * 2 <= sms && k * 2 * 2 <= chunks) k *= 2;
+  }
+  return k;
+}
+
+// One flat bf16 decode step with the unit kernel (one launch).
+mp_status unit_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* prm, void* scratch,
+                      size_t scratch_bytes, float scale, cudaStream_t st) {
+  const mp_config& c = idx->cfg;
+  if (scratch_bytes < unit_scratch_bytes(c, idx->slots)) return MP_ENOSPC;
+  const int U = c.batch * c.kv_heads, G = c.q_heads / c.kv_heads, D = c.head_dim;
+  unit::Args a{};
+  const void* Kp = ws_ptr(idx, S_KP);
+  const void* Vp = ws_ptr(idx, S_VP);
+  if (!encode_tiles(&a.tmA, ws_ptr(idx, S_KC), (uint64_t)U * idx->slots, D, unit::kRows) ||
+      !encode_tiles(&a.tmB, ws_ptr(idx, S_VC), (uint64_t)U * idx->slots, D, unit::kRows) ||
+      !encode_boxes(&a.tmKV, Kp, Vp, (uint64_t)U * c.max_tokens, D))
+    return MP_ECUDA;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.off = static_cast<const int32_t*>(ws_ptr(idx, S_OFF));
+  a.S = static_cast<float*>(scratch);
+  a.sel_mask_out = prm->sel_mask_out;
+  a.scores_out = prm->scores_out;
+  a.err = err_word(idx);
+  a.units = U;
+  a.rows = idx->slots;
+  const int64_t blocks_used = (idx->n_clustered + c.block_tokens - 1) / c.block_tokens;
+  a.rows_active = (int)std::min<int64_t>(idx->slots, blocks_used * idx->slots_per_block);
+  a.max_tokens = c.max_tokens;
+  a.n_clustered = (int)idx->n_clustered;
+  a.n_tail = (int)(idx->n_tokens - idx->n_clustered);
+  a.scale = scale;
+  a.budget = prm->budget;
+  a.approx = (prm->flags & MP_NO_APPROX) == 0;
+  a.timeout_ns = 2000000000LL;
+  a.k = cluster_size(U, (a.rows_active + unit::kRows - 1) / unit::kRows, prm->n_split);
+
+  auto phase = [&](int i) {
+    if (i < prm->n_phase_events && prm->phase_events[i])
+      cudaEventRecord(static_cast<cudaEvent_t>(prm->phase_events[i]), st);
+  };
+  phase(0);
+  cudaError_t e = launch_unit<unit::M_FLAT>(D, G, a, st);
+  phase(1);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MP_ECUDA;
+  }
+  return MP_OK;
+}
+
+// Dense decode over a plain cache: every key of [0, n) of each head exact.
+mp_status dense_decode_impl(const mp_config& c, const void* K, const void* V, int n, const void* Q, void* O,
+                            float scale, cudaStream_t st) {
+  const int U = c.batch * c.kv_heads, G = c.q_heads / c.kv_heads, D = c.head_dim;
+  unit::Args a{};
+  if (!encode_tiles(&a.tmA, K, (uint64_t)U * c.max_tokens, D, unit::kDRows) ||
+      !encode_tiles(&a.tmB, V, (uint64_t)U * c.max_tokens, D, unit::kDRows))
+    return MP_ECUDA;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.units = U;
+  a.rows = c.max_tokens;
+  a.rows_active = n;
+  a.max_tokens = c.max_tokens;
+  a.scale = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  a.approx = 0;
+  a.timeout_ns = 2000000000LL;
+  a.k = cluster_size(U, (n + unit::kDRows - 1) / unit::kDRows, 0);
+  cudaError_t e = launch_unit<unit::M_DENSE>(D, G, a, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MP_ECUDA;
+  }
+  return MP_OK;
+}
+
+}  // namespace mp

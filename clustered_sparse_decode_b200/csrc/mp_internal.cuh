@@ -28,14 +28,9 @@ enum DeviceError : int32_t {
   E_BAD_LIST = 2,       // an internal run list inconsistent with its header
   E_TIMEOUT = 4,        // a bounded wait gave up
   E_CAPACITY = 8,       // a per-unit limit of a kernel was exceeded
-  E_SCRATCH = 16,       // a ticket word of the decode scratch was not zero at the start of a step
 };
 
 constexpr int kWarp = 32;
-// The first kScratchTicketBytes of every decode scratch hold the two-pass
-// decode's ticket words (two per unit, fewer than 512 units).  The decode
-// leaves them zero; no other user of the scratch writes them.
-constexpr size_t kScratchTicketBytes = 4096;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 

@@ -30,8 +30,7 @@
  *    (e.g. corrupt offsets in an imported index) sets a device error word and
  *    skips the faulty access; mp_check_device_error reports it.  Its bits:
  *    1 a run offset or slot outside the index, 2 an inconsistent internal run
- *    list, 4 a bounded wait gave up, 8 a per-unit kernel limit exceeded,
- *    16 a decode scratch whose ticket head was not zero.
+ *    list, 4 a bounded wait gave up, 8 a per-unit kernel limit exceeded.
  *  - An index is not thread-safe: one host thread, one stream at a time.
  */
 #ifndef MPATTN_H
@@ -135,12 +134,9 @@ typedef struct {
                                scored non-empty fine cluster, -inf elsewhere */
   float* coarse_scores_out; /* optional [B, H, coarse_slots] (levels == 2) */
   void** phase_events;      /* optional: n_phase_events cudaEvent_t handles (created by the caller)
-                               recorded on `stream` at the kernel boundaries of the step, in order:
-                               flat bf16, slots <= 4096: start | ticket reset | centroid pass + value pass
-                               other flat:  start | centroid pass | select | token pass | combine
-                               levels 2:    start | coarse pass | coarse select | fine pass |
-                                            fine select | token pass | combine
-                               (3, 5 resp. 7 events; extra handles are not touched) */
+                               recorded on `stream` at the kernel boundaries of the step: the start,
+                               then the end of each phase that mp_decode_phases names for the index
+                               (extra handles are not touched) */
   int32_t n_phase_events;
   int32_t reserved2;        /* must be 0 */
 } mp_decode_params;
@@ -216,17 +212,6 @@ mp_status mp_cluster_assign(const mp_index* idx, const void* K, int32_t n, int32
 mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
                     void* d_scratch, size_t scratch_bytes, void* stream);
 
-/* The first MP_SCRATCH_TICKET_BYTES of every decode scratch hold the arrival
- * counters of the two-pass decode kernels (an implementation detail, no
- * counterpart in the paper).  They must be zero before the first mp_decode
- * that uses the buffer (e.g. one cudaMemset when it is allocated); every
- * finished decode leaves them zero, so a scratch can serve any number of
- * steps and indices without a reset.  After mp_check_device_error has
- * reported an error, zero them again (mp_decode_static_reset for the
- * library's own scratch).  A decode that finds them non-zero sets bit 16 of
- * the device error word. */
-#define MP_SCRATCH_TICKET_BYTES 4096u
-
 /* Size of the library's own decode scratch used by mp_decode_static. */
 #define MP_STATIC_SCRATCH_BYTES (32u << 20)
 
@@ -240,20 +225,23 @@ mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode
  * loads the library holds until the process exits.  It calls no allocator.
  *  - Returns MP_ENOSPC if the configuration's decode_scratch_bytes
  *    (mp_workspace_size) exceed MP_STATIC_SCRATCH_BYTES.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    A flat bf16 index needs only room for a staged Q (B * Hq * d * 2
+ *    bytes: 128 KiB at batch 16, 32 query heads, d 128), so every flat bf16
+ *    configuration up to 4096 query rows of d 128 fits; fp32 and two-level
+ *    indexes need the multi-kernel path's partials and run lists, which grow
+ *    with batch x heads x slots.
+ *  - The first call on each device, and the first after the device's current
+ *    context changed (cudaDeviceReset, another driver-API context made
+ *    current), looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current; make that first call before any stream
+ *    capture.
  *  - All calls on a device share the one array and it keeps the last call's
- *    contents; its ticket head (MP_SCRATCH_TICKET_BYTES) starts zeroed.
- *    Calls that overlap on the GPU (other streams, other threads, other
- *    indices) race on it: order them, e.g. on one stream. */
+ *    contents; every call writes what it reads, so it needs no
+ *    initialisation and no reset.  Calls that overlap on the GPU (other
+ *    streams, other threads, other indices) race on it: order them, e.g. on
+ *    one stream. */
 mp_status mp_decode_static(const mp_index* idx, const void* Q, void* O, const mp_decode_params* params,
                            void* stream);
-
-/* Zero the ticket head of the library's own decode scratch on the current
- * device (enqueued on `stream`), e.g. after mp_check_device_error reported an
- * error for a mp_decode_static call. */
-mp_status mp_decode_static_reset(void* stream);
 
 /* Device pointers of the index arrays (layouts above). */
 mp_status mp_index_export(const mp_index* idx, mp_index_view* view);
@@ -268,6 +256,26 @@ mp_status mp_index_import(mp_index* idx, const mp_index_view* src, int64_t n_tok
  * Returns MP_OK, MP_EDEVICE (word was set; *code receives it, nullable) or
  * MP_ECUDA. */
 mp_status mp_check_device_error(const mp_index* idx, int32_t* code, void* stream);
+
+/* Dense decode: exact softmax attention of every query head over all n
+ * cached keys of its KV head, no clustering.  It is the comparison point the
+ * pages measure the method against (FlashDecoding; "Multipole Attention ...",
+ * atlas.scime summary, "Key results" and "Experimental setup"), built here on
+ * the same streaming engine as mp_decode.  `cfg` gives batch, kv_heads,
+ * q_heads, head_dim, dtype and the row stride max_tokens (its clustering
+ * fields are ignored).  K, V: device [B, H, max_tokens, d]; keys [0, n) of
+ * each head are attended.  Q, O: device [B, Hq, d].  scale 0 => 1/sqrt(d).
+ * Needs no scratch and allocates nothing.  bf16 only (MP_EUNSUPPORTED
+ * otherwise); MP_EINVAL for n outside [0, max_tokens] or NULL pointers.  n = 0
+ * writes O = 0. */
+mp_status mp_dense_decode(const mp_config* cfg, const void* K, const void* V, int32_t n, const void* Q, void* O,
+                          float scale, void* stream);
+
+/* The phases of a decode step of this index, in order, separated by '|'
+ * (e.g. "decode" for the one-kernel flat bf16 path): mp_decode records
+ * phase_events[0] at the start and phase_events[i] at the end of phase i.
+ * A static string; "" for a NULL index. */
+const char* mp_decode_phases(const mp_index* idx);
 
 /* Static description of a status code. */
 const char* mp_status_str(mp_status s);

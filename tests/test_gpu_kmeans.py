@@ -431,3 +431,141 @@ def test_assign_duplicate_centroids_take_lower_slot(d, L_blk, n):
     want = oracle_assign(o, Kc, Kq, n)
     for (b, h), (ao, _, _) in want.items():
         np.testing.assert_array_equal(a[b, h], ao)
+
+
+def test_online_update_bf16_matches_oracle():
+    """The online update with bf16 keys, d 128 and 4 query heads per KV head:
+    re-clustering of the open 2048-token block assigns on the tensor cores from
+    the update's block buffer.  One Lloyd iteration per (re-)clustering, and
+    the whole index is compared after the build and after every update call:
+    while a head's state equals the oracle's, both sides start each trigger
+    from identical centroids, so the head may diverge only in rows inside the
+    fp32 tie band of those centroids; from then on it is retired.  Decoding with
+    every cluster selected is dense attention."""
+    o = H.ocfg(B=1, Hkv=2, Hq=8, d=128, n_max=8192, T=16, L_blk=2048, update_interval=512, dtype="bf16",
+               iters=1, seed=23)
+    K, V, _ = H.cache_for(o, 8192, comps=128, outliers=(4, 4.0), seed=24)
+    keys = ("Kc", "Vc", "off", "Kp", "Vp", "perm", "assign")
+
+    def same_head(ga, h, n):
+        return all(np.array_equal(ga[k][0, h], oidx[k][0, h]) for k in ("Kc", "Vc", "off")) and \
+            all(np.array_equal(ga[k][0, h, :n], oidx[k][0, h, :n]) for k in ("Kp", "Vp", "perm", "assign"))
+
+    def explained(ga, h, records, n):
+        """Every differing assignment of head h lies in a block re-clustered now, inside the tie band."""
+        diff = np.nonzero(ga["assign"][0, h, :n] != oidx["assign"][0, h, :n])[0]
+        if diff.size == 0:
+            return False
+        for (b, hh, j, X, ini, hist) in records:
+            if hh != h:
+                continue
+            rows = diff[(diff >= j * 2048) & (diff < j * 2048 + X.shape[0])] - j * 2048
+            band = band_for(X, ini)
+            if not np.all(hist[0]["gap"][rows] <= band[rows]):
+                return False
+            diff = np.setdiff1d(diff, rows + j * 2048)
+        return diff.size == 0
+
+    prompt = 3000
+    rec_b = {}
+    oidx = mp.build_index(K, V, prompt, o, record=rec_b)
+    g = gpu_build(o, K, V, prompt)
+    ga = arrays_np(g)
+    live = set()
+    for h in range(2):
+        if same_head(ga, h, prompt):
+            live.add(h)
+        else:
+            recs = []
+            for j in range(2):
+                X = K[0, h, j * 2048:min(prompt, (j + 1) * 2048)].astype(np.float64)
+                C = -(-X.shape[0] // 16)
+                recs.append((0, h, j, X, X[mp.kmeanspp_pick(X, C, mp.stream_uniforms(23, h, j, 0, C))],
+                             rec_b[(0, h, j)]))
+            assert explained(ga, h, recs, prompt), f"head {h} differs after the build outside the tie band"
+    pos = prompt
+    fired = compared = 0
+    for step in [300, 212, 1, 1000, 600, 2000]:
+        rec = []
+        f_o = mp.cluster_update(oidx, K[:, :, pos:pos + step], V[:, :, pos:pos + step], record=rec)
+        f_g = g.update(H.tdev(K[:, :, pos:pos + step], "bf16"), H.tdev(V[:, :, pos:pos + step], "bf16"))
+        assert f_o == f_g
+        fired += f_g
+        pos += step
+        assert g.n_tokens == oidx["n_tokens"] and g.n_clustered == oidx["n_clustered"]
+        torch.cuda.synchronize()
+        ga = arrays_np(g)
+        for h in sorted(live):
+            if same_head(ga, h, pos):
+                compared += f_g
+                continue
+            assert f_g and explained(ga, h, rec, pos), f"head {h} differs after an update outside the tie band"
+            live.discard(h)
+    assert g.check_device_error() == 0
+    assert fired >= 3
+    assert compared >= 2, "fewer than two re-clusterings were compared bit for bit"
+    check_invariants(o, ga, K, V, oidx["n_clustered"])
+    Q = synth.make_queries(1, 1, 8, 128, "bf16", seed=4)[0]
+    O_g = H.to_np(g.decode(H.tdev(Q, "bf16"), 1 << 20))
+    assert np.abs(O_g - mp.dense_attention(Q, K, V, pos, 2)).max() <= H.TOL["bf16"]
+
+
+def test_full_size_build_sampled_blocks():
+    """The default bench workload's build at full size: batch 16 x 8 KV heads x
+    32768 tokens, 4 blocks of 8192 keys per head, 512 centroids per block, 10
+    Lloyd iterations from k-means++ seeds, bf16 keys (tensor-core assignment).
+    Eight sampled (unit, block) pairs follow the oracle's trajectory: the GPU
+    builds with 1 .. 10 iterations match it bit for bit (assignment,
+    centroids, offsets) until an iteration in which every differing row lies
+    inside the fp32 tie band of the centroids both sides then hold.  The
+    sampled heads also satisfy the index invariants."""
+    w = synth.workload("batch16_32k_sparse95")
+    B, Hk, n, d, Lb, T = w["B"], w["Hkv"], w["n"], w["d"], w["L_blk"], w["T"]
+    o = H.ocfg(B=B, Hkv=Hk, Hq=w["Hq"], d=d, n_max=n, T=T, L_blk=Lb, iters=w["iters"], dtype="bf16", seed=w["seed"])
+    K, V, _ = synth.make_cache(B, Hk, n, d, w["comps"], w["sigma"], radius=w["radius"], outliers=w["outliers"],
+                               dtype="bf16", seed=w["seed"])
+    Kd, Vd = H.tdev(K, "bf16"), H.tdev(V, "bf16")
+    C = Lb // T
+    samples = [(0, 0, 0), (1, 3, 2), (5, 7, 1), (7, 2, 3), (9, 5, 0), (12, 1, 2), (14, 6, 3), (15, 4, 1)]
+    traj = {}
+    for (b, h, j) in samples:
+        X = K[b, h, j * Lb:(j + 1) * Lb].astype(np.float64)
+        init = X[mp.kmeanspp_pick(X, C, mp.stream_uniforms(w["seed"], b * Hk + h, j, 0, C))]
+        _, _, hist = mp.lloyd(X, init, w["iters"], "bf16")
+        traj[(b, h, j)] = (X, init, hist)
+    following = set(samples)
+    exact_to_end = 0
+    for k in range(1, w["iters"] + 1):
+        g = MultipoleIndex(H.gcfg(dict(o, iters=k)))
+        g.build(Kd, Vd)
+        torch.cuda.synchronize()
+        assert g.check_device_error() == 0
+        arr = g.arrays()
+        for (b, h, j) in sorted(following):
+            X, init, hist = traj[(b, h, j)]
+            sl = slice(j * C, (j + 1) * C)
+            a_g = arr["assign"][b, h, j * Lb:(j + 1) * Lb].cpu().numpy().astype(np.int64) - j * C
+            a_o = hist[k - 1]["assign"]
+            diff = np.nonzero(a_g != a_o)[0]
+            if diff.size == 0:
+                np.testing.assert_array_equal(H.to_np(arr["Kc"][b, h, sl]), hist[k - 1]["cents"],
+                                              err_msg=f"Kc {(b, h, j, k)}")
+                off = arr["off"][b, h, j * C:(j + 1) * C + 1].cpu().numpy().astype(np.int64)
+                np.testing.assert_array_equal(np.diff(off), np.bincount(a_o, minlength=C), err_msg=f"off {(b, h, j, k)}")
+                if k == w["iters"]:
+                    exact_to_end += 1
+                continue
+            prev = hist[k - 2]["cents"] if k >= 2 else init
+            band = band_for(X, prev)
+            assert np.all(hist[k - 1]["gap"][diff] <= band[diff]), \
+                f"block {(b, h, j)} iteration {k}: assignments differ outside the fp32 tie band"
+            following.discard((b, h, j))
+        if k == w["iters"]:
+            ga = {key: arr[key][[s[0] for s in samples], [s[1] for s in samples]] for key in ("Kc", "Vc", "off", "Kp", "Vp", "perm", "assign")}
+            ga = {key: (H.to_np(v) if v.dtype in (torch.bfloat16, torch.float32) else v.cpu().numpy().astype(np.int64))[:, None]
+                  for key, v in ga.items()}
+            Ks = np.stack([K[b, h] for (b, h, _) in samples])[:, None]
+            Vs = np.stack([V[b, h] for (b, h, _) in samples])[:, None]
+            check_invariants(dict(o, B=len(samples), Hkv=1), ga, Ks, Vs, n)
+        del g, arr
+    assert exact_to_end >= 1, "no sampled block stayed bit-exact through all iterations"

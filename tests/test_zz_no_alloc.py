@@ -37,12 +37,13 @@ def test_static_scratch_decode_matches_decode(dtype, levels):
 
 
 def test_static_scratch_rejects_configurations_that_do_not_fit():
+    # an fp32 index decodes on the multi-kernel path, whose partials grow with batch x heads
     cfg = Config(batch=32, kv_heads=8, q_heads=64, head_dim=128, max_tokens=256, block_tokens=256,
-                 kmeans_iters=1, dtype="bf16")
+                 kmeans_iters=1, dtype="f32")
     _, scratch = __import__("clustered_sparse_decode_b200").workspace_size(cfg)
     assert scratch > L.MP_STATIC_SCRATCH_BYTES
     idx = MultipoleIndex(cfg)
-    Q = torch.zeros((32, 64, 128), dtype=torch.bfloat16, device="cuda")
+    Q = torch.zeros((32, 64, 128), dtype=torch.float32, device="cuda")
     with pytest.raises(MpError) as e:
         idx.decode_static(Q, 16)
     assert e.value.status == L.MP_ENOSPC
@@ -52,9 +53,9 @@ def test_static_scratch_rejects_configurations_that_do_not_fit():
 
 
 def test_one_scratch_serves_indices_of_different_shapes():
-    """The library's array serves, in turn, two-pass indices of 4 and 16 units
-    and a multi-kernel (fp32) index, many steps each: the ticket head stays
-    zero between steps (no error bit, results equal to mp_decode's)."""
+    """The library's array serves, in turn, flat bf16 indices of 4 and 16
+    units and a multi-kernel (fp32) index, many steps each, whatever the
+    previous call left in it (no error bit, results equal to mp_decode's)."""
     shapes = [("bf16", 2, 2), ("bf16", 4, 4), ("f32", 2, 2)]
     runs = []
     for s, (dtype, B, Hkv) in enumerate(shapes):

@@ -9,8 +9,8 @@
 // cluster enters the same softmax as one term with logit score + ln(size) and
 // its value centroid.
 //
-// Per unit, in one CTA (or cluster), every load of the cache by TMA:
-//   1. key centroids    128-row tiles of Kc: scores S[c][g] = scale q_g.Kc_c
+// Per unit, in one CTA (or cluster):
+//   1. key centroids    128-row TMA tiles of Kc: scores S[c][g] = scale q_g.Kc_c
 //                       (to the scratch, each read back by the thread that
 //                       wrote it or after a block barrier) and group scores
 //                       max_g S[c][g] (shared memory).
@@ -18,27 +18,27 @@
 //                       (a cluster first gathers its CTAs' scores over
 //                       distributed shared memory): clusters in descending
 //                       score, ties to the lower slot, the crossing cluster
-//                       whole.  Meanwhile the producer already streams 3.:
-//                       its loads do not depend on the selection.
-//   3. value centroids  128-row tiles of Vc: the centroid terms of the
+//                       whole.  Meanwhile the loaders already stream 3.: its
+//                       loads do not depend on the selection.
+//   3. value centroids  128-row TMA tiles of Vc: the centroid terms of the
 //                       UNSELECTED non-empty clusters (logit S + ln n_c, value
 //                       Vc_c) enter the online softmax; selected clusters are
 //                       masked, so no term is ever added and taken out again.
 //   4. exact rows       the selected clusters' runs of the cluster-ordered
-//                       store, then the un-clustered tail, as 8-row boxes of
-//                       keys and values (one TMA each).  A run's last partial
-//                       box is placed to end at the run's end, overlapping the
-//                       run's previous box, and is issued one ring later, when
-//                       the overlapping rows are already in L2: DRAM reads each
-//                       row of the run once.
+//                       store, then the un-clustered tail, packed 64 rows to a
+//                       chunk: the planner warp lists the rows in order, the
+//                       loader warps gather them (keys and values, 16-byte
+//                       cp.async into the swizzled 8-row box layout), so every
+//                       selected row is read once and no row is padding.
 //   5. combine          the eight warps' softmax states (and, in a cluster,
 //                       the CTAs' states over distributed shared memory)
 //                       merge into O.
 //
 // Warps: 8 compute warps in two groups of 4; group w computes the chunks
 // k = w (mod 2) of a ring of 32 KB chunks (d = 128), on mma.sync (bf16 in, fp32
-// accumulate); one producer warp fills the ring.  Every wait on the device is
-// bounded (then an error bit is set and the kernel winds down).
+// accumulate); loader warp w fills the ring slots of group w's chunks; one
+// planner warp turns the selection into the row list.  Every wait on the
+// device is bounded (then an error bit is set and the kernel winds down).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -54,27 +54,30 @@ using namespace sc;
 constexpr int kCW = 8;                         // compute warps (two groups of 4)
 constexpr int kCT = kCW * kWarp;               // compute threads
 constexpr int kGW = 4;                         // warps per compute group
-constexpr int kThreads = kCT + kWarp;          // + one producer warp
+constexpr int kThreads = kCT + 2 * kWarp;      // + the loader warp and the planner warp
 constexpr int kRows = 128;                     // centroid rows per chunk (keys or values only)
 constexpr int kDRows = 64;                     // dense chunks: key and value rows
-constexpr int kBoxes = 8;                      // 8-row boxes (keys and values) per exact chunk
+constexpr int kChunkRows = 64;                 // exact rows (keys and values) per chunk, as 8-row boxes
+constexpr int kBoxes = kChunkRows / 8;
 constexpr int kMaxNS = 12;                     // ring slots at most
 constexpr int kMinNS = 4;
 constexpr int kMaxSpt = 16;                    // selection: slots per compute thread
 constexpr int kMaxSlots = kMaxSpt * kCT;       // 4096
 constexpr int kMaxCluster = 8;
-constexpr int kSegCap = 64;                    // producer run queue: segments ...
-constexpr int kTailCap = 256;                  // ... and tail boxes waiting for their release
+constexpr int kRowCap = 1024;                  // planner -> loaders: packed exact rows in flight
+constexpr int kFullCount = kGW * kWarp;        // arrivals completing a full slot: one per thread of its group
 constexpr int kSmemLimit = 232448;             // dynamic shared memory of one CTA per SM
 constexpr int kBarC = 2;                       // named barrier: compute threads
+constexpr int kBarG0 = 3;                      // named barriers 3, 4: the threads of compute group 0, 1
 
 enum Mode : int { M_FLAT = 0, M_DENSE = 1 };
-enum ChunkKind : int { K_KC = 0, K_VC = 1, K_BOX = 2, K_DENSE = 3, K_END = 4 };
+enum ChunkKind : int { K_KC = 0, K_VC = 1, K_DENSE = 2 };
 
 struct Args {
   CUtensorMap tmA;             // M_FLAT: Kc, M_DENSE: K, as [units*rows][D] bf16, 64-column tiles (128-byte swizzle)
   CUtensorMap tmB;             // M_FLAT: Vc, M_DENSE: V
-  CUtensorMap tmKV;            // M_FLAT: Kp and Vp as one map (columns, rows, [half,] key/value): 8-row boxes
+  const char* Kp;              // M_FLAT: cluster-ordered key store [units * max_tokens][D] bf16
+  const char* Vp;              // M_FLAT: value store, same layout
   const __nv_bfloat16* Q;      // [units][G][D]
   __nv_bfloat16* O;            // [units][G][D]
   const int32_t* off;          // M_FLAT: [units][slots + 1]
@@ -93,16 +96,15 @@ struct Args {
 };
 
 // What the producer tells the compute warps about the chunk in a ring slot.
-struct Meta {
-  int kind, cnt, p0, pad;      // cnt: rows (K_KC, K_VC, K_DENSE) or boxes (K_BOX); p0: first row
-  uint8_t lo[kBoxes], hi[kBoxes];   // K_BOX: valid rows [lo, hi) of each box
-  int row[kBoxes];             // K_BOX: first store row of each box (tensor-map row coordinate)
+struct Meta {                  // (tile chunks only; exact chunks need none)
+  int kind, cnt, p0, pad;      // cnt: valid rows; p0: first row
 };
-constexpr int kMetaBytes = 64;
+constexpr int kMetaBytes = 16;
 static_assert(sizeof(Meta) <= kMetaBytes, "meta");
 
-// A ring slot holds kRows centroid rows, kBoxes exact 8-row boxes (keys and
-// values) or kDRows dense rows (keys and values): 256 D bytes.
+// A ring slot holds kRows centroid rows, kChunkRows exact rows (keys and
+// values, as 8-row boxes: [box][key/value][64-column half][8 rows][128 B]) or
+// kDRows dense rows (keys and values): 256 D bytes.
 template <int D>
 struct Geo {
   static constexpr int SLOT = kRows * D * 2;
@@ -124,7 +126,7 @@ __host__ __device__ inline void plan(Args& a, int mode, int slots, int G) {
   const int offs = mode == M_FLAT ? r16((sc + 1) * 4) : 0;
   const int selm = mode == M_FLAT ? r16(sc / 8) : 0;
   const int wpre = mode == M_FLAT ? r16((sc / 32 + 1) * 4) : 0;
-  const int q = mode == M_FLAT ? kSegCap * 8 + kTailCap * 16 : 0;
+  const int q = mode == M_FLAT ? kRowCap * 4 + 16 : 0;
   const int red = mode == M_FLAT ? 1024 * 4 : 0;
   const int bar = 2 * kMaxNS * 8 + 16;
   const int fixed = meta + shat + offs + selm + wpre + q + red + bar;
@@ -182,6 +184,19 @@ __device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
   return v;
 }
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync %0, %1;\n" ::"n"(kBarC), "n"(kCT) : "memory"); }
+// barrier of n threads on named barrier id with the AND / OR of p over them
+__device__ __forceinline__ bool bar_and(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n bar.red.and.pred b, %2, %3, a;\n selp.u32 %0, 1, 0, b;\n}\n"
+               : "=r"(r) : "r"((uint32_t)p), "r"(id), "r"(n) : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool bar_or(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n bar.red.or.pred b, %2, %3, a;\n selp.u32 %0, 1, 0, b;\n}\n"
+               : "=r"(r) : "r"((uint32_t)p), "r"(id), "r"(n) : "memory");
+  return r != 0;
+}
 
 // ---------------------------------------------------------------------------
 // Selection over the group scores (compute threads).  Token-budgeted:
@@ -192,30 +207,53 @@ __device__ __forceinline__ void cbar() { asm volatile("bar.sync %0, %1;\n" ::"n"
 // W(key >= tau) >= budget, keys being the order-preserving uint32 images of
 // the group scores) is found first through 256 equal-width score bins (when at
 // most 32 clusters fall into the crossing bin one warp sorts them), else by a
-// radix descent over 256-bin histograms of the keys.  shat: [slots] group
-// scores; writes the bitmask selm (complete after the final barrier).
+// radix descent over 256-bin histograms of the keys.  Every pass reads the
+// scores and counts from shared memory in rolled loops: the selection runs
+// once per step, so its code is kept small.  shat: [slots] group scores;
+// writes the bitmask selm (complete after the final barrier).
 // ---------------------------------------------------------------------------
+// warp 0: the first of 256 bins (8 per lane, bin 8 l + i) from the top whose
+// running weight, counted from `base` above, reaches the budget; the weight
+// strictly above that bin.  Results in red[0], red[1].
+__device__ __forceinline__ void crossing_bin(const int* hist, int base, int budget, int lane, int* red) {
+  int bl[8], ls = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { bl[i] = hist[8 * lane + i]; ls += bl[i]; }
+  int suf = ls;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  int run = base + suf - ls, found = -1, ab = 0;
+#pragma unroll
+  for (int i = 7; i >= 0; --i) {
+    if (found < 0 && run + bl[i] >= budget) { found = 8 * lane + i; ab = run; }
+    run += bl[i];
+  }
+  const unsigned m = __ballot_sync(kFull, found >= 0);
+  const int src = 31 - __clz(m);
+  const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
+  if (lane == 0) { red[0] = fb; red[1] = fa; }
+}
+
 template <int G>
 __device__ void select_smem(const Args& a, const float* shat, const int32_t* offs, uint32_t* selm, int* red,
                             int* hist, int u, bool write_out) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int slots = a.rows_active;
-  // thread tid owns slots tid + k kCT: a warp reads 32 consecutive slots (no
-  // bank conflicts) and the selection of 32 consecutive slots is one ballot
-  uint32_t key[kMaxSpt];
-  int w[kMaxSpt];
+  // 1. total weight, smallest and largest key of the non-empty clusters
   int wsum = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-#pragma unroll
-  for (int k = 0; k < kMaxSpt; ++k) {
-    const int c = tid + k * kCT;
-    const bool in = c < slots;
-    const int cnt = in ? offs[c + 1] - offs[c] : 0;
-    const float sh = cnt > 0 ? shat[c] : -INFINITY;
-    key[k] = cnt > 0 ? ordered_key(sh) : 0u;
-    w[k] = cnt > 0 ? cnt : 0;
-    wsum += w[k];
-    if (cnt > 0) { kmin = min(kmin, key[k]); kmax = max(kmax, key[k]); }
+#pragma unroll 1
+  for (int c = tid; c < slots; c += kCT) {
+    const int w = offs[c + 1] - offs[c];
+    if (w > 0) {
+      const uint32_t kk = ordered_key(shat[c]);
+      wsum += w;
+      kmin = min(kmin, kk);
+      kmax = max(kmax, kk);
+    }
   }
   {
     const int ws_ = __reduce_add_sync(kFull, wsum);
@@ -237,6 +275,7 @@ __device__ void select_smem(const Args& a, const float* shat, const int32_t* off
   int ntie = 0, above = 0;
   bool resolved = false;
   if (mode == 2) {
+    // 2a. 256 equal-width score bins; the crossing bin's clusters, if at most 32, sorted by one warp
     const float smin = key_score(kmin), smax = key_score(kmax);
     const float span = smax - smin, inv = 256.f / span;
     if (isfinite(smin) && isfinite(smax) && span > 0.f && isfinite(span) && isfinite(inv)) {
@@ -245,67 +284,47 @@ __device__ void select_smem(const Args& a, const float* shat, const int32_t* off
       for (int i = tid; i < 256; i += kCT) hist[i] = 0;
       if (tid == 0) red[3] = 0;
       cbar();
-#pragma unroll
-      for (int k = 0; k < kMaxSpt; ++k)
-        if (w[k] > 0) atomicAdd(hist + fbin(key[k]), w[k]);
-      cbar();
-      if (warp == 0) {
-        int bl[8], ls = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { bl[i] = hist[8 * lane + i]; ls += bl[i]; }
-        int suf = ls;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_down_sync(kFull, suf, o);
-          if (lane + o < 32) suf += y;
-        }
-        int run = suf - ls, found = -1, ab = 0;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          if (found < 0 && run + bl[i] >= a.budget) { found = 8 * lane + i; ab = run; }
-          run += bl[i];
-        }
-        const unsigned m = __ballot_sync(kFull, found >= 0);
-        const int src = 31 - __clz(m);
-        const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
-        if (lane == 0) { red[0] = fb; red[1] = fa; }
+#pragma unroll 1
+      for (int c = tid; c < slots; c += kCT) {
+        const int w = offs[c + 1] - offs[c];
+        if (w > 0) atomicAdd(hist + fbin(ordered_key(shat[c])), w);
       }
       cbar();
+      if (warp == 0) crossing_bin(hist, 0, a.budget, lane, red);
+      cbar();
       const int fb = red[0], ab = red[1];
-#pragma unroll
-      for (int k = 0; k < kMaxSpt; ++k)
-        if (w[k] > 0 && fbin(key[k]) == fb) {
-          const int pos = atomicAdd(red + 3, 1);
-          if (pos < 32) { lst[3 * pos] = (int)key[k]; lst[3 * pos + 1] = tid + k * kCT; lst[3 * pos + 2] = w[k]; }
+#pragma unroll 1
+      for (int c = tid; c < slots; c += kCT) {
+        const int w = offs[c + 1] - offs[c];
+        if (w > 0) {
+          const uint32_t kk = ordered_key(shat[c]);
+          if (fbin(kk) == fb) {
+            const int pos = atomicAdd(red + 3, 1);
+            if (pos < 32) { lst[3 * pos] = (int)kk; lst[3 * pos + 1] = c; lst[3 * pos + 2] = w; }
+          }
         }
+      }
       cbar();
       const int nc = red[3];
       if (nc <= 32) {
         if (warp == 0) {
-          // lane l holds candidate l; empty lanes sort last with weight 0
-          uint64_t v = lane < nc ? ((uint64_t)(uint32_t)lst[3 * lane] << 32) | (uint32_t)(0xffffffffu - (uint32_t)lst[3 * lane + 1])
-                                 : 0ull;
-          int wl = lane < nc ? lst[3 * lane + 2] : 0;
-#pragma unroll
-          for (int kk = 2; kk <= 32; kk <<= 1) {
-#pragma unroll
-            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-              const uint64_t ov = __shfl_xor_sync(kFull, v, jj);
-              const int ow = __shfl_xor_sync(kFull, wl, jj);
-              const bool up = ((lane & kk) == 0) == ((lane & jj) == 0);   // this lane keeps the larger
-              if (up ? ov > v : ov < v) { v = ov; wl = ow; }
-            }
+          // lane l holds candidate l (key, weight); the crossing key t is the
+          // largest key whose candidates at or above it bring the running
+          // weight ab + W(key >= t) to the budget
+          const uint32_t kl = lane < nc ? (uint32_t)lst[3 * lane] : 0u;
+          const int wl = lane < nc ? lst[3 * lane + 2] : 0;
+          int wgt = 0, weq = 0;
+#pragma unroll 1
+          for (int j = 0; j < nc; ++j) {
+            const uint32_t kj = (uint32_t)__shfl_sync(kFull, (int)kl, j);
+            const int wj = __shfl_sync(kFull, wl, j);
+            wgt += kj > kl ? wj : 0;
+            weq += kj == kl ? wj : 0;
           }
-          int inc = wl;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, inc, o);
-            if (lane >= o) inc += y;
-          }
-          const unsigned cross = __ballot_sync(kFull, lane < nc && ab + inc >= a.budget);
-          const uint32_t t = (uint32_t)(__shfl_sync(kFull, v, __ffs(cross) - 1) >> 32);
-          const uint32_t kl = (uint32_t)(v >> 32);
-          const int gt = __reduce_add_sync(kFull, lane < nc && kl > t ? wl : 0);
+          const bool reach = lane < nc && ab + wgt + weq >= a.budget;
+          const uint32_t t = __reduce_max_sync(kFull, reach ? kl : 0u);
+          const int tl = __ffs(__ballot_sync(kFull, reach && kl == t)) - 1;
+          const int gt = __shfl_sync(kFull, wgt, tl);
           const int nt = __popc(__ballot_sync(kFull, lane < nc && kl == t));
           if (lane == 0) { red[0] = (int)t; red[1] = ab + gt; red[2] = nt; }
         }
@@ -319,112 +338,100 @@ __device__ void select_smem(const Args& a, const float* shat, const int32_t* off
     }
   }
   if (mode == 2 && !resolved) {
+    // 2b. radix descent over the keys in [kmin, kmax], 8 bits at a time
     uint32_t lo = kmin;
     int nb = kmax == kmin ? 0 : 32 - __clz(kmax - kmin);
     above = 0;
     int* hcnt = hist + 256;
     ntie = -1;
+#pragma unroll 1
     while (nb > 0) {
       const int sh = max(nb - 8, 0);
       for (int i = tid; i < 256; i += kCT) { hist[i] = 0; hcnt[i] = 0; }
       cbar();
       const unsigned long long hi_excl = (unsigned long long)lo + (1ull << nb);
-#pragma unroll
-      for (int k = 0; k < kMaxSpt; ++k)
-        if (w[k] > 0 && key[k] >= lo && (unsigned long long)key[k] < hi_excl) {
-          const int bin = (int)((key[k] - lo) >> sh);
-          atomicAdd(hist + bin, w[k]);
-          if (sh == 0) atomicAdd(hcnt + bin, 1);
+#pragma unroll 1
+      for (int c = tid; c < slots; c += kCT) {
+        const int w = offs[c + 1] - offs[c];
+        if (w > 0) {
+          const uint32_t kk = ordered_key(shat[c]);
+          if (kk >= lo && (unsigned long long)kk < hi_excl) {
+            const int bin = (int)((kk - lo) >> sh);
+            atomicAdd(hist + bin, w);
+            if (sh == 0) atomicAdd(hcnt + bin, 1);
+          }
         }
-      cbar();
-      if (warp == 0) {
-        int bl[8], ls = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { bl[i] = hist[8 * lane + i]; ls += bl[i]; }
-        int suf = ls;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_down_sync(kFull, suf, o);
-          if (lane + o < 32) suf += y;
-        }
-        int run = above + suf - ls;
-        int found = -1, ab = 0;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          if (found < 0 && run + bl[i] >= a.budget) { found = 8 * lane + i; ab = run; }
-          run += bl[i];
-        }
-        const unsigned m = __ballot_sync(kFull, found >= 0);
-        const int src = 31 - __clz(m);
-        const int fb = __shfl_sync(kFull, found, src), fa = __shfl_sync(kFull, ab, src);
-        if (lane == 0) { red[0] = fb; red[1] = fa; red[2] = hcnt[fb]; }
       }
       cbar();
-      const int b = red[0];
+      if (warp == 0) {
+        crossing_bin(hist, above, a.budget, lane, red);
+        __syncwarp();
+        if (lane == 0) red[2] = hcnt[red[0]];
+      }
+      cbar();
+      const int bsel = red[0];
       above = red[1];
       if (sh == 0) ntie = red[2];
-      lo += (uint32_t)b << sh;
+      lo += (uint32_t)bsel << sh;
       nb = sh;
       cbar();
     }
     tau = lo;
   }
-  const int need = mode == 2 ? a.budget - above : 0;   // tokens still to take among the ties at tau
-  // several clusters exactly at tau: they are taken in slot order, slot tid + k kCT
-  // after every slot of rows k' < k and of lower threads in row k
-  int tie_before[kMaxSpt];
-#pragma unroll
-  for (int k = 0; k < kMaxSpt; ++k) tie_before[k] = 0;
-  if (mode == 2 && ntie != 1) {
-    int row_base = 0;
-#pragma unroll
-    for (int k = 0; k < kMaxSpt; ++k) {
-      const int tw = (key[k] == tau && w[k] > 0) ? w[k] : 0;
-      int inc = tw;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, inc, o);
-        if (lane >= o) inc += y;
-      }
-      if (lane == 31) red[64 + warp] = inc;
-      cbar();
-      int pre = 0, row = 0;
-#pragma unroll
-      for (int i = 0; i < kCW; ++i) {
-        pre += i < warp ? red[64 + i] : 0;
-        row += red[64 + i];
-      }
-      tie_before[k] = row_base + pre + inc - tw;
-      row_base += row;
-      cbar();
-    }
-  }
-  // the selection of slots [32 (8 k + warp), + 32): one ballot, one word
-#pragma unroll
-  for (int k = 0; k < kMaxSpt; ++k) {
+  // 3. the selection bits: every cluster above tau, and the one at tau when
+  // no other cluster ties with it (it is the crossing cluster: always taken)
+#pragma unroll 1
+  for (int base = warp * 32; base < slots; base += kCT) {
+    const int c = base + lane;
     bool sel = false;
-    if (w[k] > 0) {
-      if (mode == 1) sel = true;
-      else if (mode == 2) sel = key[k] > tau || (key[k] == tau && tie_before[k] < need);
+    if (c < slots && offs[c + 1] > offs[c]) {
+      if (mode == 1) {
+        sel = true;
+      } else if (mode == 2) {
+        const uint32_t kk = ordered_key(shat[c]);
+        sel = kk > tau || (ntie == 1 && kk == tau);
+      }
     }
     const unsigned bits = __ballot_sync(kFull, sel);
-    if (lane == 0 && k * kCT + warp * 32 < slots) selm[k * kCW + warp] = bits;
-    if (write_out) {
-      const int c = tid + k * kCT;
-      if (c < slots) {
-        if (a.sel_mask_out) a.sel_mask_out[(size_t)u * a.rows + c] = sel ? 1 : 0;
-        if (a.scores_out) a.scores_out[(size_t)u * a.rows + c] = w[k] > 0 ? key_score(key[k]) : -INFINITY;
-      }
-    }
-  }
-  if (write_out) {
-    // slots of blocks that hold no tokens yet
-    for (int c = slots + tid; c < a.rows; c += kCT) {
-      if (a.sel_mask_out) a.sel_mask_out[(size_t)u * a.rows + c] = 0;
-      if (a.scores_out) a.scores_out[(size_t)u * a.rows + c] = -INFINITY;
-    }
+    if (lane == 0) selm[base >> 5] = bits;
   }
   cbar();
+  if (mode == 2 && ntie != 1) {
+    // several clusters exactly at tau: taken in slot order while the tokens
+    // taken among them stay below budget - above (one warp; ties are rare)
+    if (warp == 0) {
+      const int need = a.budget - above;
+      int taken = 0;
+#pragma unroll 1
+      for (int base = 0; base < slots && taken < need; base += 32) {
+        const int c = base + lane;
+        int tw = 0;
+        if (c < slots) {
+          const int w = offs[c + 1] - offs[c];
+          if (w > 0 && ordered_key(shat[c]) == tau) tw = w;
+        }
+        int inc = tw;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const unsigned bits = __ballot_sync(kFull, tw > 0 && taken + inc - tw < need);
+        if (lane == 0 && bits) selm[base >> 5] |= bits;
+        taken += __shfl_sync(kFull, inc, 31);
+      }
+    }
+    cbar();
+  }
+  if (write_out) {
+#pragma unroll 1
+    for (int c = tid; c < a.rows; c += kCT) {
+      const bool in = c < slots && offs[c + 1] > offs[c];
+      const bool sel = c < slots && ((selm[c >> 5] >> (c & 31)) & 1u);
+      if (a.sel_mask_out) a.sel_mask_out[(size_t)u * a.rows + c] = sel ? 1 : 0;
+      if (a.scores_out) a.scores_out[(size_t)u * a.rows + c] = in ? shat[c] : -INFINITY;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -459,76 +466,76 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      mbar_init(full0 + 8 * i, 1);           // the producer's arrival (+ the TMA bytes it announces)
+      mbar_init(full0 + 8 * i, kFullCount);  // the loader's arrivals (+ the TMA bytes it announces)
       mbar_init(empty0 + 8 * i, kGW);        // one arrival per warp of the chunk's compute group
     }
     mbar_init(selready, 1);                  // the selection is in shared memory
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    if (MODE == M_FLAT) {
+      volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
+      ctl[0] = 0;
+      ctl[1] = -1;
+      ctl[2] = 0;
+      ctl[3] = 0;
+    }
   }
+  __syncthreads();
   if (MODE == M_FLAT && warp < kCW) {
-    // the unit's run offsets (counts of every slot), for the centroid terms and the selection
+    // the unit's run offsets (counts of every slot), for the centroid terms and the
+    // selection: complete for every compute thread after the selection's first barrier
     const int32_t* ou = a.off + (size_t)u * (a.rows + 1);
     for (int i = threadIdx.x; i <= a.rows_active; i += kCT) offs[i] = __ldg(ou + i);
   }
-  __syncthreads();
 
-  if (warp == kCW) {
-    // ============================ producer ============================
-    int k = 0;              // chunk counter (all streams)
-    bool ok = true;
-    auto acquire = [&](int kk) -> bool {   // wait until the slot of chunk kk is free
-      const int slot = kk % NS;
-      bool got = true;
-      if (kk >= NS && lane == 0) got = mbar_wait(empty0 + 8 * slot, ((kk / NS) - 1) & 1, deadline);
-      got = __shfl_sync(kFull, got ? 1 : 0, 0) != 0;
-      if (!got && lane == 0) set_error(a.err, E_TIMEOUT);
-      return got;
-    };
-    // ---- first stream: key centroid tiles (flat) or key and value tiles (dense) ----
-    for (int x = c_lo; x < c_hi && ok; ++x, ++k) {
-      if (!(ok = acquire(k))) break;
-      const int slot = k % NS;
-      if (lane == 0) {
-        Meta* m = meta(slot);
-        const int p0 = x * CR;
-        m->kind = MODE == M_FLAT ? K_KC : K_DENSE;
-        m->cnt = min(CR, a.rows_active - p0);
-        m->p0 = p0;
-        const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
-        const int y = u * a.rows + p0;
-        mbar_arrive_tx(bar, (uint32_t)Gm::SLOT);
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_2d(dst + h * (CR * 128), &a.tmA, 64 * h, y, bar);
-        if (MODE == M_DENSE) {
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h) tma_2d(dst + Gm::DAREA + h * (CR * 128), &a.tmB, 64 * h, y, bar);
+  if (warp >= kCW) {
+    // ========================= loader and planner =========================
+    int32_t* rowq = reinterpret_cast<int32_t*>(smem + a.o_q);                    // packed exact rows
+    volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
+    // ctl[0]: rows published, ctl[1]: all rows (-1 until known), ctl[2 + g]: compute
+    // group g has read every row queue entry below 64 ctl[2 + g]
+    if (K > 1 && MODE == M_FLAT) cluster_arrive();   // (1): nothing of these warps' is read by the peers
+    if (warp == kCW) {
+      // ---------------- loader: every TMA tile chunk ----------------
+      // key centroid tiles (flat) or key and value tiles (dense), then value
+      // centroid tiles; the exact rows are gathered by the compute groups
+      const int kx0 = MODE == M_FLAT && a.approx ? 2 * n1 : n1;
+      for (int k = 0; k < kx0; ++k) {
+        const int slot = k % NS;
+        bool got = true;
+        if (k >= NS && lane == 0) got = mbar_wait(empty0 + 8 * slot, ((k / NS) - 1) & 1, deadline);
+        if (!__shfl_sync(kFull, got ? 1 : 0, 0)) {
+          if (lane == 0) set_error(a.err, E_TIMEOUT);
+          break;
         }
-      }
-    }
-    if constexpr (MODE == M_FLAT) {
-      if (K > 1) cluster_arrive();         // (1): nothing of this warp's is read by the peers
-      // ---- value centroid tiles: their loads do not wait for the selection ----
-      if (a.approx) {
-        for (int x = c_lo; x < c_hi && ok; ++x, ++k) {
-          if (!(ok = acquire(k))) break;
-          const int slot = k % NS;
-          if (lane == 0) {
-            Meta* m = meta(slot);
-            const int p0 = x * kRows;
-            m->kind = K_VC;
-            m->cnt = min(kRows, a.rows_active - p0);
-            m->p0 = p0;
-            const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
-            mbar_arrive_tx(bar, (uint32_t)Gm::SLOT);
+        if (lane == 0) {
+          Meta* m = meta(slot);
+          const bool vc = k >= n1;
+          const int p0 = (c_lo + (vc ? k - n1 : k)) * CR;
+          m->kind = MODE == M_FLAT ? (vc ? K_VC : K_KC) : K_DENSE;
+          m->cnt = min(CR, a.rows_active - p0);
+          m->p0 = p0;
+          const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
+          const int y = u * a.rows + p0;
+          mbar_expect_tx(bar, (uint32_t)Gm::SLOT);
+          const CUtensorMap* tm = vc ? &a.tmB : &a.tmA;
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) tma_2d(dst + h * (kRows * 128), &a.tmB, 64 * h, u * a.rows + p0, bar);
+          for (int h = 0; h < D / 64; ++h) tma_2d(dst + h * (CR * 128), tm, 64 * h, y, bar);
+          if (MODE == M_DENSE) {
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) tma_2d(dst + Gm::DAREA + h * (CR * 128), &a.tmB, 64 * h, y, bar);
           }
+          mbar_arrive_cnt(bar, kFullCount);
         }
+        __syncwarp();
       }
-      // ---- exact rows: needs the selection ----
-      bool got = true;
-      if (lane == 0) got = mbar_wait(selready, 0, deadline);
-      if (!__shfl_sync(kFull, got ? 1 : 0, 0)) {
+    } else if constexpr (MODE == M_FLAT) {
+      // ---------------- planner ----------------
+      // Walks the selection in slot order and packs the rows of the selected
+      // clusters' runs, then this CTA's share of the un-clustered tail, into
+      // the row queue (rows of the key and value stores, one entry per row).
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(selready, 0, deadline);
+      if (!__shfl_sync(kFull, ok ? 1 : 0, 0)) {
         if (lane == 0) set_error(a.err, E_TIMEOUT);
         ok = false;
       }
@@ -554,47 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
       const int t_lo = a.n_clustered + (int)((long long)rank * a.n_tail / K);
       const int t_hi = a.n_clustered + (int)((long long)(rank + 1) * a.n_tail / K);
       const int unit_row = u * a.max_tokens;
-      const int zero_row = a.units * a.max_tokens;   // a box wholly past the stores: zero-filled, no reads
-      const int DM = kBoxes * NS;                    // a tail box waits this many main boxes: one ring
-      // Run queue: segments {first row, full boxes (> 0) | -(rows of a run under 8 rows)}
-      // and tail boxes {first row, first valid row, release (main boxes issued), 0}.
-      int2* segq = reinterpret_cast<int2*>(smem + a.o_q);
-      int4* tailq = reinterpret_cast<int4*>(smem + a.o_q + kSegCap * 8);
-      int sh = 0, stl = 0, th = 0, ttl = 0;          // ring heads and tails (monotone, warp-uniform)
-      int rk = r_lo, seg_off = 0;                    // next rank to enqueue; boxes of the head segment issued
-      bool tail_run = t_lo < t_hi;                   // the un-clustered tail still to enqueue
-      long long mb_enq = 0, mb_iss = 0;              // main boxes enqueued / issued
-      // enqueue one run per lane (valid lanes): its full boxes as a segment, its
-      // last < 8 rows as a tail box ending at the run's end, released one ring later
-      auto enqueue = [&](bool valid, int st, int cnt) {
-        const int nf = cnt >> 3, rem = cnt & 7;
-        const unsigned vm = __ballot_sync(kFull, valid);
-        const unsigned lt = (1u << lane) - 1u;
-        if (valid) segq[(stl + __popc(vm & lt)) % kSegCap] = make_int2(st, nf > 0 ? nf : -cnt);
-        int mb = valid ? (nf > 0 ? nf : 1) : 0, inc = mb;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(kFull, inc, o);
-          if (lane >= o) inc += y;
-        }
-        const bool tl = valid && nf > 0 && rem > 0;
-        const unsigned tm = __ballot_sync(kFull, tl);
-        if (tl)
-          tailq[(ttl + __popc(tm & lt)) % kTailCap] =
-              make_int4(st + cnt - 8, 8 - rem, (int)(mb_enq + inc + DM), 0);
-        stl += __popc(vm);
-        ttl += __popc(tm);
-        mb_enq += __shfl_sync(kFull, inc, 31);
-      };
-      // the next up to 32 selected clusters, one per lane, located by rank
-      auto refill = [&]() {
+      int written = 0;
+      bool tail_run = t_lo < t_hi;
+      for (int rk = r_lo; ok && (rk < r_hi || tail_run);) {
+        // up to 32 runs, one per lane: selected clusters located by rank, or the tail
+        int st = 0, cnt = 0;
         if (rk < r_hi) {
           const int n = min(32, r_hi - rk);
-          bool valid = false;
-          int st = 0, cnt = 0;
           if (lane < n) {
             const int r = rk + lane;
-            int lo = 0, hi = nw - 1;                 // the word holding rank r: the last w with wpre[w] <= r
+            int lo = 0, hi = nw - 1;             // the word holding rank r: the last w with wpre[w] <= r
             while (lo < hi) {
               const int mid = (lo + hi + 1) >> 1;
               if (wpre[mid] <= r) lo = mid; else hi = mid - 1;
@@ -607,118 +583,60 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
               const int sl = (lo << 5) + __ffs(word) - 1;
               st = offs[sl];
               cnt = offs[sl + 1] - st;
-              if (st < 0 || cnt < 1 || st + cnt > a.max_tokens) set_error(a.err, E_BAD_OFFSET);
-              else valid = true;
+              if (st < 0 || cnt < 1 || st + cnt > a.max_tokens) {
+                set_error(a.err, E_BAD_OFFSET);
+                cnt = 0;
+              }
             }
           }
-          enqueue(valid, st, cnt);
           rk += n;
-        } else if (tail_run) {
-          enqueue(lane == 0, t_lo, t_hi - t_lo);
+        } else {
+          if (lane == 0) { st = t_lo; cnt = t_hi - t_lo; }
           tail_run = false;
         }
-      };
-      for (;;) {
-        // keep at least one chunk of segments queued (while the tail-box ring has room)
-        while ((rk < r_hi || tail_run) && stl - sh < kBoxes && ttl - th <= kTailCap - 32) refill();
-        const bool done_enq = rk >= r_hi && !tail_run;
-        if (!ok || (sh == stl && th == ttl && done_enq)) break;
-        if (!(ok = acquire(k))) break;
-        const int slot = k % NS;
-        Meta* m = meta(slot);
-        // lane-parallel assembly: lane b < kBoxes works out box b of the chunk.
-        // First the tail boxes whose runs' full boxes were issued one ring ago
-        // (the rows they share with those boxes are in L2 by now), in release
-        // order; then main boxes from the next segments.
-        const unsigned lo8 = (1u << kBoxes) - 1u;
-        int4 tv = make_int4(0, 0, 0, 0);
-        const bool has_t = lane < kBoxes && th + lane < ttl;
-        if (has_t) tv = tailq[(th + lane) % kTailCap];
-        int nt = __ffs(~(__ballot_sync(kFull, has_t && tv.z <= mb_iss) & lo8)) - 1;   // released prefix
-        int2 sg = make_int2(0, 0);
-        int sb_cnt = 0;                          // boxes left in segment sh + lane
-        if (lane < kBoxes && sh + lane < stl) {
-          sg = segq[(sh + lane) % kSegCap];
-          sb_cnt = (sg.y > 0 ? sg.y : 1) - (lane == 0 ? seg_off : 0);
-        }
-        int incl = sb_cnt;
+        int incl = cnt;
 #pragma unroll
-        for (int o = 1; o < kBoxes; o <<= 1) {
+        for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(kFull, incl, o);
           if (lane >= o) incl += y;
         }
-        const int avail = __shfl_sync(kFull, incl, kBoxes - 1);
-        int nm = min(kBoxes - nt, avail);        // main boxes in this chunk
-        if (nm == 0) {
-          // no main box left (or none queued): waiting tail boxes go now
-          nt = min(kBoxes, ttl - th);
-        } else if (sh + kBoxes >= stl && done_enq && nm == avail) {
-          // the last main boxes: released or not, tail boxes fill the chunk
-          nt = min(kBoxes - nm, ttl - th);
-        }
-        int row = 0, blo = 0, bhi = 0;
-        bool on = false;
-        if (lane < nt) {
-          row = unit_row + tv.x;
-          blo = tv.y;
-          bhi = 8;
-          on = true;
-        }
-        const int mi = lane - nt;                // main box number in this chunk
-        // segment of main box mi: the first lane j with incl_j > mi
-        int seg_j = 0;
+        const int nrows = __shfl_sync(kFull, incl, 31);
+        for (int b0 = 0; b0 < nrows; b0 += 32) {
+          // room for 32 more entries: the loaders have taken every row below 64 min(next chunk)
+          bool room = true;
+          if (lane == 0) {
+            for (;;) {
+              const int lo_j = min(ctl[2], ctl[3]);
+              if (written + b0 + 32 - kChunkRows * lo_j <= kRowCap) break;
+              if (gtimer() > deadline) { room = false; break; }
+              __nanosleep(64);
+            }
+          }
+          if (!__shfl_sync(kFull, room ? 1 : 0, 0)) {
+            if (lane == 0) set_error(a.err, E_TIMEOUT);
+            ok = false;
+            break;
+          }
+          // entry b0 + lane lies in the run of the first lane whose inclusive count exceeds it
+          const int q = b0 + lane;
+          int lo = 0, hi = 31;
 #pragma unroll
-        for (int jj = 0; jj < kBoxes; ++jj) seg_j += (__shfl_sync(kFull, incl, jj) <= mi) ? 1 : 0;
-        const int incl_prev = __shfl_sync(kFull, incl, max(seg_j - 1, 0));   // every lane takes part
-        const int before = seg_j > 0 ? incl_prev : 0;
-        const int2 sj = make_int2(__shfl_sync(kFull, sg.x, min(seg_j, kBoxes - 1)),
-                                  __shfl_sync(kFull, sg.y, min(seg_j, kBoxes - 1)));
-        if (lane < kBoxes && mi >= 0 && mi < nm) {
-          const int off_in = mi - before + (seg_j == 0 ? seg_off : 0);
-          if (sj.y > 0) { row = unit_row + sj.x + 8 * off_in; blo = 0; bhi = 8; }
-          else { row = unit_row + sj.x; blo = 0; bhi = -sj.y; }   // a run under 8 rows: the rows after it are masked
-          on = true;
+          for (int step = 0; step < 5; ++step) {
+            const int mid = (lo + hi) >> 1;
+            if (__shfl_sync(kFull, incl, mid) > q) hi = mid; else lo = mid + 1;
+          }
+          const int before = __shfl_sync(kFull, incl - cnt, lo);
+          const int rs = __shfl_sync(kFull, st, lo);
+          if (q < nrows) rowq[(written + q) % kRowCap] = unit_row + rs + (q - before);
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) ctl[0] = written + min(b0 + 32, nrows);
         }
-        int nb = nt + nm;
-        if ((nb & 1) && lane == nb) { row = zero_row; blo = 0; bhi = 0; on = true; }   // all-zero partner box
-        nb += nb & 1;
-        if (on) {
-          m->lo[lane] = (uint8_t)blo;
-          m->hi[lane] = (uint8_t)bhi;
-          m->row[lane] = row;
-        }
-        // advance the queues past this chunk's boxes
-        {
-          const int full_segs = __popc(__ballot_sync(kFull, lane < kBoxes && sb_cnt > 0 && incl <= nm) & lo8);
-          const int incl_last = __shfl_sync(kFull, incl, max(full_segs - 1, 0));   // every lane takes part
-          const int used = full_segs > 0 ? incl_last : 0;
-          seg_off = full_segs > 0 ? nm - used : seg_off + nm;
-          sh += full_segs;
-          th += nt;
-          mb_iss += nm;
-        }
-        if (lane == 0) {
-          m->kind = K_BOX;
-          m->cnt = nb;
-        }
-        __syncwarp();
-        const uint32_t dst = sb + slot * Gm::SLOT, bar = full0 + 8 * slot;
-        if (lane == 0) mbar_arrive_tx(bar, (uint32_t)(nb * Gm::BOXB));
-        __syncwarp();
-        if (lane < nb) tma_box<D>(dst + lane * Gm::BOXB, &a.tmKV, row, bar);
-        ++k;
+        written += nrows;
       }
-    }
-    // end markers: one for each compute group
-    for (int e = 0; e < 2 && ok; ++e, ++k) {
-      if (!(ok = acquire(k))) break;
-      const int slot = k % NS;
-      if (lane == 0) {
-        meta(slot)->kind = K_END;
-        meta(slot)->cnt = 0;
-        mbar_arrive(full0 + 8 * slot);
-      }
+      __threadfence_block();
       __syncwarp();
+      if (lane == 0) ctl[1] = ok ? written : 0;
     }
     if (K > 1) {
       if (MODE == M_FLAT) cluster_wait();  // (1)
@@ -816,76 +734,160 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
     if (threadIdx.x == 0) mbar_arrive(selready);   // the producer may walk the selection
   }
   // ---- value centroids and exact rows ----
-  for (int k = n1 + ((grp - n1) % 2 + 2) % 2; alive; k += 2) {
-    // a value-centroid chunk: its scores come from the scratch (written by the
-    // key stream before the selection's barriers); load them before the wait
-    float sv[2][2][2];
-    const bool vc_chunk = MODE == M_FLAT && a.approx && k < 2 * n1;
-    if (vc_chunk) {
-      const int p0 = (c_lo + k - n1) * kRows;
+  // A value-centroid chunk's scores come from the scratch (written by the key
+  // stream before the selection's barriers): each group loads them one of its
+  // chunks ahead, so that the loads overlap the previous chunk.
+  auto load_sv = [&](int kk, float (&sv)[2][2][2]) {
+    if (!(MODE == M_FLAT && a.approx && kk < 2 * n1)) return;
+    const int p0 = (c_lo + kk - n1) * kRows;
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = p0 + wg * 32 + t * 16 + WarpSoftmax<D, G>::zrow(lane, i);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int h = WarpSoftmax<D, G>::col_head(lane, j);
+          sv[t][i][j] = (h >= 0 && r < a.rows_active) ? __ldcg(a.S + ((size_t)u * a.rows + r) * SG + h) : 0.f;
+        }
+      }
+  };
+  if constexpr (MODE == M_FLAT) {
+    // Exact chunk c (c >= kx0, packed rows [64 j, 64 j + 64), j = c - kx0) is
+    // gathered by the group that computes it, into its slot, once the group
+    // has consumed the slot's previous chunk c - NS and the planner has
+    // published the rows.  Decisions are group-uniform: every thread reads the
+    // planner's counters itself and a barrier reduction combines them.
+    volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
+    const int32_t* rowq = reinterpret_cast<const int32_t*>(smem + a.o_q);
+    const int kx0 = a.approx ? 2 * n1 : n1;
+    const int gbar = kBarG0 + grp, gt = threadIdx.x - grp * kGW * kWarp;
+    int nxt = kx0 + ((grp - kx0) % 2 + 2) % 2;    // this group's next exact chunk to gather
+    int kend = 0x7fffffff;                        // this group's first chunk past the rows
+    // gathers this group's exact chunks while their slots are free (c < k + NS
+    // once chunk k - 2 is consumed) and their rows published; with `must`,
+    // waits until chunk k itself is gathered or known to lie past the rows
+    auto gather = [&](int k, bool must) -> bool {
+      while (nxt < kend && nxt < k + NS) {
+        const int j = nxt - kx0;
+        const int total = ctl[1], avail = ctl[0];
+        const bool ready = total >= 0 || avail >= kChunkRows * (j + 1);
+        if (!bar_and(gbar, kGW * kWarp, ready)) {
+          if (!must || nxt != k) return true;     // try again at the next chunk
+          if (bar_or(gbar, kGW * kWarp, gtimer() > deadline)) {
+            if (gt == 0) set_error(a.err, E_TIMEOUT);
+            return false;
+          }
+          __nanosleep(64);
+          continue;
+        }
+        __threadfence_block();                    // the published rows, after their count
+        if (total >= 0 && kChunkRows * j >= total) {
+          kend = nxt;
+          return true;
+        }
+        const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * j) : kChunkRows;
+        const int q0 = kChunkRows * j;
+        const uint32_t dst = sb + (nxt % NS) * Gm::SLOT;
+        if constexpr (D == 128) {
+          // one row (keys and values, 2 x 256 B) per warp instruction: lane = kv:1 half:1 c16:3
+          const int kv = lane >> 4, half = (lane >> 3) & 1, c16 = lane & 7;
+          const char* g = (kv ? a.Vp : a.Kp) + half * 128 + c16 * 16;
+          const uint32_t d0 = dst + kv * (Gm::BOXB / 2) + half * (Gm::BOXB / 4);
+#pragma unroll 4
+          for (int s2 = 0; s2 < kChunkRows / kGW; ++s2) {
+            const int i = kGW * s2 + wg, rr = i & 7;
+            const bool v = i < cnt;
+            const int r = v ? rowq[(q0 + i) % kRowCap] : 0;
+            cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)r * 256, v);
+          }
+        } else {
+          // two rows (keys and values, 2 x 128 B each) per warp instruction: lane = row:1 kv:1 c16:3
+          const int sub = lane >> 4, kv = (lane >> 3) & 1, c16 = lane & 7;
+          const char* g = (kv ? a.Vp : a.Kp) + c16 * 16;
+          const uint32_t d0 = dst + kv * (Gm::BOXB / 2);
+#pragma unroll 4
+          for (int s2 = 0; s2 < kChunkRows / (2 * kGW); ++s2) {
+            const int i = 2 * (kGW * s2 + wg) + sub, rr = i & 7;
+            const bool v = i < cnt;
+            const int r = v ? rowq[(q0 + i) % kRowCap] : 0;
+            cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)r * 128, v);
+          }
+        }
+        cp_arrive_noinc(full0 + 8 * (nxt % NS));   // one of the slot's 128 arrivals, once this thread's copies land
+        if (gt == 0) ctl[2 + grp] = j;           // the group's earlier chunks' entries are read
+        nxt += 2;
+      }
+      return true;
+    };
+    float sv[2][2][2], svn[2][2][2];
+    const int k2 = n1 + ((grp - n1) % 2 + 2) % 2;   // this group's first chunk of the second stream
+    load_sv(k2, sv);
+    for (int k = k2; alive; k += 2) {
+      if (!gather(k, k >= kx0)) {
+        alive = false;
+        break;
+      }
+      if (k >= kend) break;
+      load_sv(k + 2, svn);
+      if (!wait_full(k)) break;
+      const int slot = k % NS;
+      const uint32_t base = sb + slot * Gm::SLOT;
+      if (k < kx0) {
+        // value centroids of the unselected non-empty clusters: logit S + ln n
+        const Meta* m = meta(slot);
+        const int cnt = m->cnt, p0 = m->p0;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int r16 = wg * 32 + t * 16;
+          if (r16 < cnt) {
+            float z[2][2];
+            bool any = false;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
+              const int s = p0 + r;
+              const int n = r < cnt ? offs[s + 1] - offs[s] : 0;
+              const bool take = n > 0 && !((selm[s >> 5] >> (s & 31)) & 1u);
+              const float lg = log2f((float)n);
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const int h = WarpSoftmax<D, G>::col_head(lane, j);
+                z[i][j] = (take && h >= 0) ? sv[t][i][j] * kLog2e + lg : -INFINITY;
+                any |= take && h >= 0;
+              }
+            }
+            if (__any_sync(kFull, any)) ws.template update<false, kRows>(base, r16, lane, z, 1.f);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * slot);   // the loader may refill the slot
+      } else {
+        // exact rows: the chunk's valid rows follow from the planner's counters
+        const int j = k - kx0, total = ctl[1];
+        const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * j) : kChunkRows;
+        const int r16 = wg * 16;
+        if (r16 < cnt) {
+          float z[2][2];
+          ws.template qk<true, kRows>(base, r16, lane, z);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int r = r16 + 8 * i + (lane >> 2);   // rows 8 i .. 8 i + 7 of this warp's tile are box 2 wg + i
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+              z[i][jj] = (WarpSoftmax<D, G>::col_head(lane, jj) >= 0 && r < cnt) ? z[i][jj] * qk2 : -INFINITY;
+          }
+          ws.template update<true, kRows>(base + Gm::BOXB / 2, r16, lane, z, 1.f);
+        }
+      }
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = p0 + wg * 32 + t * 16 + WarpSoftmax<D, G>::zrow(lane, i);
+        for (int i = 0; i < 2; ++i)
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int h = WarpSoftmax<D, G>::col_head(lane, j);
-            sv[t][i][j] = (h >= 0 && r < a.rows_active) ? __ldcg(a.S + ((size_t)u * a.rows + r) * SG + h) : 0.f;
-          }
-        }
+          for (int jj = 0; jj < 2; ++jj) sv[t][i][jj] = svn[t][i][jj];
     }
-    if (!wait_full(k)) break;
-    const int slot = k % NS;
-    const Meta* m = meta(slot);
-    const int kind = m->kind, cnt = m->cnt;
-    if (kind == K_END) break;
-    const uint32_t base = sb + slot * Gm::SLOT;
-    if (kind == K_VC) {
-      // value centroids of the unselected non-empty clusters: logit S + ln n
-      const int p0 = m->p0;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int r16 = wg * 32 + t * 16;
-        if (r16 < cnt) {
-          float z[2][2];
-          bool any = false;
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int r = r16 + WarpSoftmax<D, G>::zrow(lane, i);
-            const int s = p0 + r;
-            const int n = r < cnt ? offs[s + 1] - offs[s] : 0;
-            const bool take = n > 0 && !((selm[s >> 5] >> (s & 31)) & 1u);
-            const float lg = log2f((float)n);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int h = WarpSoftmax<D, G>::col_head(lane, j);
-              z[i][j] = (take && h >= 0) ? sv[t][i][j] * kLog2e + lg : -INFINITY;
-              any |= take && h >= 0;
-            }
-          }
-          if (__any_sync(kFull, any)) ws.template update<false, kRows>(base, r16, lane, z, 1.f);
-        }
-      }
-    } else if (kind == K_BOX) {
-      const int r16 = wg * 16;
-      if (2 * wg < cnt) {
-        float z[2][2];
-        ws.template qk<true, kRows>(base, r16, lane, z);
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int bx = 2 * wg + i;            // rows 8 i .. 8 i + 7 of this warp's tile are box bx
-          const int blo = m->lo[bx], bhi = m->hi[bx];
-          const int rb = lane >> 2;
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            z[i][j] = (WarpSoftmax<D, G>::col_head(lane, j) >= 0 && rb >= blo && rb < bhi) ? z[i][j] * qk2 : -INFINITY;
-        }
-        ws.template update<true, kRows>(base + Gm::BOXB / 2, r16, lane, z, 1.f);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+    cp_wait_all();                           // this thread's gathers have landed (also on an error path)
   }
   // ---- combine ----
   cbar();                                  // every chunk is consumed: the ring is free
@@ -1013,32 +1015,6 @@ static bool encode_tiles(CUtensorMap* tm, const void* base, uint64_t rows, int D
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Kp and Vp ([rows][D] bf16 each, Vp after Kp) as one map whose outermost
-// dimension steps from Kp to Vp: an 8-row box lands as [key/value][64-column
-// half][8 rows][128 bytes], 128-byte swizzle.  The map covers exactly the two
-// stores; box rows past them read as zeros.
-static bool encode_boxes(CUtensorMap* tm, const void* Kp, const void* Vp, uint64_t rows, int D) {
-  auto fn = unit_encoder();
-  if (!fn) return false;
-  const intptr_t kv = reinterpret_cast<const char*>(Vp) - reinterpret_cast<const char*>(Kp);
-  if (kv < (intptr_t)(rows * D * 2) || (kv & 15) != 0 || kv >= ((intptr_t)1 << 40)) return false;
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  if (D == 128) {
-    cuuint64_t gdim[4] = {64, rows, 2, 2};
-    cuuint64_t gstride[3] = {256, 128, (cuuint64_t)kv};
-    cuuint32_t box[4] = {64, 8, 2, 2};
-    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(Kp), gdim, gstride, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-  }
-  cuuint64_t gdim[3] = {64, rows, 2};
-  cuuint64_t gstride[2] = {128, (cuuint64_t)kv};
-  cuuint32_t box[3] = {64, 8, 2};
-  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(Kp), gdim, gstride, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int G, int MODE>
 static cudaError_t launch_unit_t(unit::Args& a, cudaStream_t st) {
   auto kern = unit::unit_decode<D, G, MODE>;
@@ -1111,12 +1087,11 @@ mp_status unit_decode(const mp_index* idx, const void* Q, void* O, const mp_deco
   if (scratch_bytes < unit_scratch_bytes(c, idx->slots)) return MP_ENOSPC;
   const int U = c.batch * c.kv_heads, G = c.q_heads / c.kv_heads, D = c.head_dim;
   unit::Args a{};
-  const void* Kp = ws_ptr(idx, S_KP);
-  const void* Vp = ws_ptr(idx, S_VP);
   if (!encode_tiles(&a.tmA, ws_ptr(idx, S_KC), (uint64_t)U * idx->slots, D, unit::kRows) ||
-      !encode_tiles(&a.tmB, ws_ptr(idx, S_VC), (uint64_t)U * idx->slots, D, unit::kRows) ||
-      !encode_boxes(&a.tmKV, Kp, Vp, (uint64_t)U * c.max_tokens, D))
+      !encode_tiles(&a.tmB, ws_ptr(idx, S_VC), (uint64_t)U * idx->slots, D, unit::kRows))
     return MP_ECUDA;
+  a.Kp = static_cast<const char*>(ws_ptr(idx, S_KP));
+  a.Vp = static_cast<const char*>(ws_ptr(idx, S_VP));
   a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.O = static_cast<__nv_bfloat16*>(O);
   a.off = static_cast<const int32_t*>(ws_ptr(idx, S_OFF));

@@ -54,7 +54,9 @@ using namespace sc;
 constexpr int kCW = 8;                         // compute warps (two groups of 4)
 constexpr int kCT = kCW * kWarp;               // compute threads
 constexpr int kGW = 4;                         // warps per compute group
-constexpr int kThreads = kCT + 2 * kWarp;      // + the loader warp and the planner warp
+constexpr int kLoaders = 4;                    // loader warps
+constexpr int kThreads = kCT + (kLoaders + 1) * kWarp;   // + the loaders and the planner
+constexpr int kRowCap = 1024;                  // planner -> loaders: row queue entries
 constexpr int kRows = 128;                     // centroid rows per chunk (keys or values only)
 constexpr int kDRows = 64;                     // dense chunks: key and value rows
 constexpr int kChunkRows = 64;                 // exact rows (keys and values) per chunk, as 8-row boxes
@@ -64,11 +66,9 @@ constexpr int kMinNS = 4;
 constexpr int kMaxSpt = 16;                    // selection: slots per compute thread
 constexpr int kMaxSlots = kMaxSpt * kCT;       // 4096
 constexpr int kMaxCluster = 8;
-constexpr int kRowCap = 1024;                  // planner -> loaders: packed exact rows in flight
-constexpr int kFullCount = kGW * kWarp;        // arrivals completing a full slot: one per thread of its group
+constexpr int kFullCount = kLoaders * kWarp;   // arrivals completing a full slot: one per loader thread
 constexpr int kSmemLimit = 232448;             // dynamic shared memory of one CTA per SM
 constexpr int kBarC = 2;                       // named barrier: compute threads
-constexpr int kBarG0 = 3;                      // named barriers 3, 4: the threads of compute group 0, 1
 
 enum Mode : int { M_FLAT = 0, M_DENSE = 1 };
 enum ChunkKind : int { K_KC = 0, K_VC = 1, K_DENSE = 2 };
@@ -126,9 +126,9 @@ __host__ __device__ inline void plan(Args& a, int mode, int slots, int G) {
   const int offs = mode == M_FLAT ? r16((sc + 1) * 4) : 0;
   const int selm = mode == M_FLAT ? r16(sc / 8) : 0;
   const int wpre = mode == M_FLAT ? r16((sc / 32 + 1) * 4) : 0;
-  const int q = mode == M_FLAT ? kRowCap * 4 + 16 : 0;
+  const int q = mode == M_FLAT ? kRowCap * 4 + 128 : 0;
   const int red = mode == M_FLAT ? 1024 * 4 : 0;
-  const int bar = 2 * kMaxNS * 8 + 16;
+  const int bar = 2 * kMaxNS * 8 + 32;
   const int fixed = meta + shat + offs + selm + wpre + q + red + bar;
   // An even number of slots: chunk k goes to slot k % ns and to compute group
   // k % 2, so every slot always serves the same group, which waits for that
@@ -184,19 +184,8 @@ __device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
   return v;
 }
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync %0, %1;\n" ::"n"(kBarC), "n"(kCT) : "memory"); }
-// barrier of n threads on named barrier id with the AND / OR of p over them
-__device__ __forceinline__ bool bar_and(int id, int n, bool p) {
-  uint32_t r;
-  asm volatile("{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n bar.red.and.pred b, %2, %3, a;\n selp.u32 %0, 1, 0, b;\n}\n"
-               : "=r"(r) : "r"((uint32_t)p), "r"(id), "r"(n) : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ bool bar_or(int id, int n, bool p) {
-  uint32_t r;
-  asm volatile("{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n bar.red.or.pred b, %2, %3, a;\n selp.u32 %0, 1, 0, b;\n}\n"
-               : "=r"(r) : "r"((uint32_t)p), "r"(id), "r"(n) : "memory");
-  return r != 0;
-}
+// named barrier `id` of n threads
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
 
 // ---------------------------------------------------------------------------
 // Selection over the group scores (compute threads).  Token-budgeted:
@@ -475,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
       volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
       ctl[0] = 0;
       ctl[1] = -1;
-      ctl[2] = 0;
-      ctl[3] = 0;
+      for (int i = 0; i < kLoaders; ++i) ctl[2 + i] = 0;
+      for (int i = 0; i < kMaxNS; ++i) ctl[8 + i] = -1;   // gen[]: no exact chunk's slot handed over yet
     }
   }
   __syncthreads();
@@ -488,26 +477,35 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
   }
 
   if (warp >= kCW) {
-    // ========================= loader and planner =========================
-    int32_t* rowq = reinterpret_cast<int32_t*>(smem + a.o_q);                    // packed exact rows
+    // ======================== loaders and planner ========================
+    // Loader 0 issues every TMA tile chunk (key centroids, or dense keys and
+    // values; then value centroids).  The planner warp walks the selection in
+    // slot order and lists the rows of the selected clusters' runs, then this
+    // CTA's share of the un-clustered tail, in the row queue; the four loaders
+    // gather them, 64 to an exact chunk, loader i the 16 rows from 16 i, as
+    // 16-byte cp.async (keys and values) into the swizzled 8-row box layout.
+    // Every wait is taken by all 32 lanes of a warp: a warp whose lane 0 alone
+    // waits on an mbarrier (the other lanes parked at a later convergence
+    // point) runs its following code several times slower.
+    const int li = warp - kCW;               // 0..3: loader, 4: planner
+    const int kx0 = MODE == M_FLAT && a.approx ? 2 * n1 : n1;   // first exact chunk
+    int32_t* rowq = reinterpret_cast<int32_t*>(smem + a.o_q);
     volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
-    // ctl[0]: rows published, ctl[1]: all rows (-1 until known), ctl[2 + g]: compute
-    // group g has read every row queue entry below 64 ctl[2 + g]
+    // ctl[0]: rows published, ctl[1]: all rows (-1 until known), ctl[2 + i]: loader i has
+    // read every queue entry below 64 ctl[2 + i]
     if (K > 1 && MODE == M_FLAT) cluster_arrive();   // (1): nothing of these warps' is read by the peers
-    if (warp == kCW) {
-      // ---------------- loader: every TMA tile chunk ----------------
-      // key centroid tiles (flat) or key and value tiles (dense), then value
-      // centroid tiles; the exact rows are gathered by the compute groups
-      const int kx0 = MODE == M_FLAT && a.approx ? 2 * n1 : n1;
-      for (int k = 0; k < kx0; ++k) {
-        const int slot = k % NS;
-        bool got = true;
-        if (k >= NS && lane == 0) got = mbar_wait(empty0 + 8 * slot, ((k / NS) - 1) & 1, deadline);
-        if (!__shfl_sync(kFull, got ? 1 : 0, 0)) {
-          if (lane == 0) set_error(a.err, E_TIMEOUT);
-          break;
-        }
+    bool ok = true;
+    auto acquire = [&](int kk) -> bool {   // wait until the slot of chunk kk is free
+      const bool got = kk < NS || mbar_wait(empty0 + 8 * (kk % NS), ((kk / NS) - 1) & 1, deadline);
+      if (!got && lane == 0) set_error(a.err, E_TIMEOUT);
+      return __all_sync(kFull, got);
+    };
+    if (li == 0) {
+#pragma unroll 1
+      for (int k = 0; k < kx0 && ok; ++k) {
+        if (!(ok = acquire(k))) break;
         if (lane == 0) {
+          const int slot = k % NS;
           Meta* m = meta(slot);
           const bool vc = k >= n1;
           const int p0 = (c_lo + (vc ? k - n1 : k)) * CR;
@@ -528,115 +526,193 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
         }
         __syncwarp();
       }
-    } else if constexpr (MODE == M_FLAT) {
-      // ---------------- planner ----------------
-      // Walks the selection in slot order and packs the rows of the selected
-      // clusters' runs, then this CTA's share of the un-clustered tail, into
-      // the row queue (rows of the key and value stores, one entry per row).
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(selready, 0, deadline);
-      if (!__shfl_sync(kFull, ok ? 1 : 0, 0)) {
-        if (lane == 0) set_error(a.err, E_TIMEOUT);
-        ok = false;
-      }
-      const int nw = (a.rows_active + 31) >> 5;
-      int tot = 0;
-      for (int w0 = 0; w0 < nw; w0 += 32) {   // per-word prefix of selected-cluster counts
-        const int wi = w0 + lane;
-        const int c = wi < nw ? __popc(selm[wi]) : 0;
-        int inc = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(kFull, inc, o);
-          if (lane >= o) inc += y;
-        }
-        if (wi < nw) wpre[wi] = tot + inc - c;
-        tot += __shfl_sync(kFull, inc, 31);
-      }
-      if (lane == 0) wpre[nw] = tot;
-      __syncwarp();
-      // this CTA's share: selected clusters of rank [r_lo, r_hi), tail rows [t_lo, t_hi)
-      const int nsel = tot;
-      const int r_lo = (int)((long long)rank * nsel / K), r_hi = (int)((long long)(rank + 1) * nsel / K);
-      const int t_lo = a.n_clustered + (int)((long long)rank * a.n_tail / K);
-      const int t_hi = a.n_clustered + (int)((long long)(rank + 1) * a.n_tail / K);
-      const int unit_row = u * a.max_tokens;
-      int written = 0;
-      bool tail_run = t_lo < t_hi;
-      for (int rk = r_lo; ok && (rk < r_hi || tail_run);) {
-        // up to 32 runs, one per lane: selected clusters located by rank, or the tail
-        int st = 0, cnt = 0;
-        if (rk < r_hi) {
-          const int n = min(32, r_hi - rk);
-          if (lane < n) {
-            const int r = rk + lane;
-            int lo = 0, hi = nw - 1;             // the word holding rank r: the last w with wpre[w] <= r
-            while (lo < hi) {
-              const int mid = (lo + hi + 1) >> 1;
-              if (wpre[mid] <= r) lo = mid; else hi = mid - 1;
-            }
-            uint32_t word = selm[lo];
-            for (int i = wpre[lo]; i < r && word; ++i) word &= word - 1;
-            if (word == 0u) {
-              set_error(a.err, E_BAD_LIST);
-            } else {
-              const int sl = (lo << 5) + __ffs(word) - 1;
-              st = offs[sl];
-              cnt = offs[sl + 1] - st;
-              if (st < 0 || cnt < 1 || st + cnt > a.max_tokens) {
-                set_error(a.err, E_BAD_OFFSET);
-                cnt = 0;
-              }
-            }
+    }
+    if constexpr (MODE == M_FLAT) {
+      if (li < kLoaders) {
+        // ---------------- exact chunks (loader li) ----------------
+        // A slot's empty barrier may be waited on only one phase ahead of its
+        // last completed phase (the parity test cannot tell phases two apart).
+        // Loaders 1..3 issue no tile chunk, so for the first NS exact chunks,
+        // whose slots last held tile chunks, they take loader 0's word that the
+        // slot is free (gen[slot] = the chunk loader 0 acquired it for).
+        volatile int* gen = ctl + 8;
+#pragma unroll 1
+        for (int j = 0; ok; ++j) {
+          const int k = kx0 + j;
+          // the chunk's rows are published, or all rows are known (then possibly none left)
+          int total = -1, avail = 0;
+#pragma unroll 1
+          for (int spins = 0;; ++spins) {
+            total = __shfl_sync(kFull, ctl[1], 0);
+            avail = __shfl_sync(kFull, ctl[0], 0);
+            if (total >= 0 || avail >= kChunkRows * (j + 1)) break;
+            if ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline)) { ok = false; break; }
+            __nanosleep(64);
           }
-          rk += n;
-        } else {
-          if (lane == 0) { st = t_lo; cnt = t_hi - t_lo; }
-          tail_run = false;
-        }
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(kFull, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const int nrows = __shfl_sync(kFull, incl, 31);
-        for (int b0 = 0; b0 < nrows; b0 += 32) {
-          // room for 32 more entries: the loaders have taken every row below 64 min(next chunk)
-          bool room = true;
-          if (lane == 0) {
-            for (;;) {
-              const int lo_j = min(ctl[2], ctl[3]);
-              if (written + b0 + 32 - kChunkRows * lo_j <= kRowCap) break;
-              if (gtimer() > deadline) { room = false; break; }
-              __nanosleep(64);
-            }
-          }
-          if (!__shfl_sync(kFull, room ? 1 : 0, 0)) {
+          if (!ok) {
             if (lane == 0) set_error(a.err, E_TIMEOUT);
-            ok = false;
             break;
           }
-          // entry b0 + lane lies in the run of the first lane whose inclusive count exceeds it
-          const int q = b0 + lane;
-          int lo = 0, hi = 31;
-#pragma unroll
-          for (int step = 0; step < 5; ++step) {
-            const int mid = (lo + hi) >> 1;
-            if (__shfl_sync(kFull, incl, mid) > q) hi = mid; else lo = mid + 1;
-          }
-          const int before = __shfl_sync(kFull, incl - cnt, lo);
-          const int rs = __shfl_sync(kFull, st, lo);
-          if (q < nrows) rowq[(written + q) % kRowCap] = unit_row + rs + (q - before);
+          __threadfence_block();               // the published rows, after their count
+          if (total >= 0 && kChunkRows * j >= total) break;
+          const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * j) : kChunkRows;
+          const int i0 = 16 * li;
+          const int r = (lane < 16 && i0 + lane < cnt) ? rowq[(kChunkRows * j + i0 + lane) % kRowCap] : -1;
           __threadfence_block();
           __syncwarp();
-          if (lane == 0) ctl[0] = written + min(b0 + 32, nrows);
+          if (lane == 0) ctl[2 + li] = j + 1;  // this loader has read its entries of chunk j
+          if (li == 0 || k >= kx0 + NS) {
+            ok = acquire(k);
+            if (li == 0 && k < kx0 + NS) {
+              __syncwarp();
+              if (lane == 0) gen[k % NS] = ok ? k : -2;
+            }
+          } else {
+#pragma unroll 1
+            for (int spins = 0;; ++spins) {
+              const int g = __shfl_sync(kFull, gen[k % NS], 0);
+              if (g == k) break;
+              if (g == -2 || ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline))) { ok = false; break; }
+              __nanosleep(32);
+            }
+            if (!ok && lane == 0) set_error(a.err, E_TIMEOUT);
+          }
+          if (!ok) break;
+          const uint32_t dst = sb + (k % NS) * Gm::SLOT;
+          if constexpr (D == 128) {
+            // one row (keys and values, 2 x 256 B) per instruction: lane = kv:1 half:1 c16:3
+            const int kv = lane >> 4, half = (lane >> 3) & 1, c16 = lane & 7;
+            const char* g = (kv ? a.Vp : a.Kp) + half * 128 + c16 * 16;
+            const uint32_t d0 = dst + kv * (Gm::BOXB / 2) + half * (Gm::BOXB / 4);
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2) {
+              const int rw = __shfl_sync(kFull, r, s2);
+              const int i = i0 + s2, rr = i & 7;
+              cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)max(rw, 0) * 256, rw >= 0);
+            }
+          } else {
+            // two rows (keys and values, 2 x 128 B each) per instruction: lane = row:1 kv:1 c16:3
+            const int sub = lane >> 4, kv = (lane >> 3) & 1, c16 = lane & 7;
+            const char* g = (kv ? a.Vp : a.Kp) + c16 * 16;
+            const uint32_t d0 = dst + kv * (Gm::BOXB / 2);
+#pragma unroll
+            for (int s2 = 0; s2 < 16; s2 += 2) {
+              const int rw = __shfl_sync(kFull, r, s2 + sub);
+              const int i = i0 + s2 + sub, rr = i & 7;
+              cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)max(rw, 0) * 128, rw >= 0);
+            }
+          }
+          cp_arrive_noinc(full0 + 8 * (k % NS));   // one of the slot's 128 arrivals, once this lane's copies land
         }
-        written += nrows;
+        cp_wait_all();                         // this warp's copies have landed (also on an error path)
+      } else {
+        // ---------------- planner ----------------
+        if (!__all_sync(kFull, mbar_wait(selready, 0, deadline))) {
+          if (lane == 0) set_error(a.err, E_TIMEOUT);
+          ok = false;
+        }
+        const int nw = (a.rows_active + 31) >> 5;
+        int tot = 0;
+#pragma unroll 1
+        for (int w0 = 0; w0 < nw; w0 += 32) {   // per-word prefix of selected-cluster counts
+          const int wi = w0 + lane;
+          const int c = wi < nw ? __popc(selm[wi]) : 0;
+          int inc = c;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += y;
+          }
+          if (wi < nw) wpre[wi] = tot + inc - c;
+          tot += __shfl_sync(kFull, inc, 31);
+        }
+        __syncwarp();
+        // this CTA's share: selected clusters of rank [r_lo, r_hi), tail rows [t_lo, t_hi)
+        const int r_lo = (int)((long long)rank * tot / K), r_hi = (int)((long long)(rank + 1) * tot / K);
+        const int t_lo = a.n_clustered + (int)((long long)rank * a.n_tail / K);
+        const int t_hi = a.n_clustered + (int)((long long)(rank + 1) * a.n_tail / K);
+        const int unit_row = u * a.max_tokens;
+        int written = 0;
+        bool tail_run = t_lo < t_hi;
+#pragma unroll 1
+        for (int rk = r_lo; ok && (rk < r_hi || tail_run);) {
+          // up to 32 runs, one per lane: selected clusters located by rank, or the tail
+          int st = 0, cnt = 0;
+          if (rk < r_hi) {
+            const int n = min(32, r_hi - rk);
+            if (lane < n) {
+              const int r = rk + lane;
+              int lo = 0, hi = nw - 1;             // the word holding rank r: the last w with wpre[w] <= r
+#pragma unroll 1
+              while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (wpre[mid] <= r) lo = mid; else hi = mid - 1;
+              }
+              uint32_t word = selm[lo];
+#pragma unroll 1
+              for (int i = wpre[lo]; i < r && word; ++i) word &= word - 1;
+              if (word == 0u) {
+                set_error(a.err, E_BAD_LIST);
+              } else {
+                const int sl = (lo << 5) + __ffs(word) - 1;
+                st = offs[sl];
+                cnt = offs[sl + 1] - st;
+                if (st < 0 || cnt < 1 || st + cnt > a.max_tokens) {
+                  set_error(a.err, E_BAD_OFFSET);
+                  cnt = 0;
+                }
+              }
+            }
+            rk += n;
+          } else {
+            if (lane == 0) { st = t_lo; cnt = t_hi - t_lo; }
+            tail_run = false;
+          }
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const int nrows = __shfl_sync(kFull, incl, 31);
+#pragma unroll 1
+          for (int b0 = 0; b0 < nrows; b0 += 32) {
+            // room for 32 more entries: every loader has read the entries below 64 min(ctl[2 + i])
+#pragma unroll 1
+            for (int spins = 0;; ++spins) {
+              int lo_j = ctl[2 + (lane & 3)];
+              lo_j = min(lo_j, __shfl_xor_sync(kFull, lo_j, 1));
+              lo_j = min(lo_j, __shfl_xor_sync(kFull, lo_j, 2));
+              lo_j = __shfl_sync(kFull, lo_j, 0);
+              if (written + b0 + 32 - kChunkRows * lo_j <= kRowCap) break;
+              if ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline)) { ok = false; break; }
+              __nanosleep(64);
+            }
+            if (!ok) {
+              if (lane == 0) set_error(a.err, E_TIMEOUT);
+              break;
+            }
+            // entry b0 + lane lies in the run of the first lane whose inclusive count exceeds it
+            const int q = b0 + lane;
+            int lo = 0, hi = 31;
+#pragma unroll
+            for (int step = 0; step < 5; ++step) {
+              const int mid = (lo + hi) >> 1;
+              if (__shfl_sync(kFull, incl, mid) > q) hi = mid; else lo = mid + 1;
+            }
+            const int before = __shfl_sync(kFull, incl - cnt, lo);
+            const int rs = __shfl_sync(kFull, st, lo);
+            if (q < nrows) rowq[(written + q) % kRowCap] = unit_row + rs + (q - before);
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) ctl[0] = written + min(b0 + 32, nrows);
+          }
+          written += nrows;
+        }
+        __threadfence_block();
+        __syncwarp();
+        if (lane == 0) ctl[1] = ok ? written : 0;
       }
-      __threadfence_block();
-      __syncwarp();
-      if (lane == 0) ctl[1] = ok ? written : 0;
     }
     if (K > 1) {
       if (MODE == M_FLAT) cluster_wait();  // (1)
@@ -731,7 +807,8 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
       cbar();
     }
     select_smem<G>(a, shat, offs, selm, red, red + 256, u, rank == 0);
-    if (threadIdx.x == 0) mbar_arrive(selready);   // the producer may walk the selection
+    cbar();                                // every read of the group scores is done
+    if (threadIdx.x == 0) mbar_arrive(selready);   // the loaders may pack the selected rows (over the group scores)
   }
   // ---- value centroids and exact rows ----
   // A value-centroid chunk's scores come from the scratch (written by the key
@@ -753,82 +830,30 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
       }
   };
   if constexpr (MODE == M_FLAT) {
-    // Exact chunk c (c >= kx0, packed rows [64 j, 64 j + 64), j = c - kx0) is
-    // gathered by the group that computes it, into its slot, once the group
-    // has consumed the slot's previous chunk c - NS and the planner has
-    // published the rows.  Decisions are group-uniform: every thread reads the
-    // planner's counters itself and a barrier reduction combines them.
+    const int kx0 = a.approx ? 2 * n1 : n1;         // first exact chunk
     volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
-    const int32_t* rowq = reinterpret_cast<const int32_t*>(smem + a.o_q);
-    const int kx0 = a.approx ? 2 * n1 : n1;
-    const int gbar = kBarG0 + grp, gt = threadIdx.x - grp * kGW * kWarp;
-    int nxt = kx0 + ((grp - kx0) % 2 + 2) % 2;    // this group's next exact chunk to gather
-    int kend = 0x7fffffff;                        // this group's first chunk past the rows
-    // gathers this group's exact chunks while their slots are free (c < k + NS
-    // once chunk k - 2 is consumed) and their rows published; with `must`,
-    // waits until chunk k itself is gathered or known to lie past the rows
-    auto gather = [&](int k, bool must) -> bool {
-      while (nxt < kend && nxt < k + NS) {
-        const int j = nxt - kx0;
-        const int total = ctl[1], avail = ctl[0];
-        const bool ready = total >= 0 || avail >= kChunkRows * (j + 1);
-        if (!bar_and(gbar, kGW * kWarp, ready)) {
-          if (!must || nxt != k) return true;     // try again at the next chunk
-          if (bar_or(gbar, kGW * kWarp, gtimer() > deadline)) {
-            if (gt == 0) set_error(a.err, E_TIMEOUT);
-            return false;
-          }
-          __nanosleep(64);
-          continue;
-        }
-        __threadfence_block();                    // the published rows, after their count
-        if (total >= 0 && kChunkRows * j >= total) {
-          kend = nxt;
-          return true;
-        }
-        const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * j) : kChunkRows;
-        const int q0 = kChunkRows * j;
-        const uint32_t dst = sb + (nxt % NS) * Gm::SLOT;
-        if constexpr (D == 128) {
-          // one row (keys and values, 2 x 256 B) per warp instruction: lane = kv:1 half:1 c16:3
-          const int kv = lane >> 4, half = (lane >> 3) & 1, c16 = lane & 7;
-          const char* g = (kv ? a.Vp : a.Kp) + half * 128 + c16 * 16;
-          const uint32_t d0 = dst + kv * (Gm::BOXB / 2) + half * (Gm::BOXB / 4);
-#pragma unroll 4
-          for (int s2 = 0; s2 < kChunkRows / kGW; ++s2) {
-            const int i = kGW * s2 + wg, rr = i & 7;
-            const bool v = i < cnt;
-            const int r = v ? rowq[(q0 + i) % kRowCap] : 0;
-            cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)r * 256, v);
-          }
-        } else {
-          // two rows (keys and values, 2 x 128 B each) per warp instruction: lane = row:1 kv:1 c16:3
-          const int sub = lane >> 4, kv = (lane >> 3) & 1, c16 = lane & 7;
-          const char* g = (kv ? a.Vp : a.Kp) + c16 * 16;
-          const uint32_t d0 = dst + kv * (Gm::BOXB / 2);
-#pragma unroll 4
-          for (int s2 = 0; s2 < kChunkRows / (2 * kGW); ++s2) {
-            const int i = 2 * (kGW * s2 + wg) + sub, rr = i & 7;
-            const bool v = i < cnt;
-            const int r = v ? rowq[(q0 + i) % kRowCap] : 0;
-            cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)r * 128, v);
-          }
-        }
-        cp_arrive_noinc(full0 + 8 * (nxt % NS));   // one of the slot's 128 arrivals, once this thread's copies land
-        if (gt == 0) ctl[2 + grp] = j;           // the group's earlier chunks' entries are read
-        nxt += 2;
-      }
-      return true;
-    };
     float sv[2][2][2], svn[2][2][2];
     const int k2 = n1 + ((grp - n1) % 2 + 2) % 2;   // this group's first chunk of the second stream
     load_sv(k2, sv);
     for (int k = k2; alive; k += 2) {
-      if (!gather(k, k >= kx0)) {
-        alive = false;
-        break;
+      if (k >= kx0) {
+        // exact chunk j exists once the planner has published a row of it; none is
+        // left once all rows are known and they end before it
+        const int j = k - kx0;
+        int total = -1;
+#pragma unroll 1
+        for (int spins = 0;; ++spins) {
+          total = ctl[1];
+          if (total >= 0 || ctl[0] > kChunkRows * j) break;
+          if ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline)) {
+            if (lane == 0) set_error(a.err, E_TIMEOUT);
+            alive = false;
+            break;
+          }
+          __nanosleep(64);
+        }
+        if (!alive || (total >= 0 && kChunkRows * j >= total)) break;
       }
-      if (k >= kend) break;
       load_sv(k + 2, svn);
       if (!wait_full(k)) break;
       const int slot = k % NS;
@@ -860,12 +885,10 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
             if (__any_sync(kFull, any)) ws.template update<false, kRows>(base, r16, lane, z, 1.f);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * slot);   // the loader may refill the slot
       } else {
-        // exact rows: the chunk's valid rows follow from the planner's counters
-        const int j = k - kx0, total = ctl[1];
-        const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * j) : kChunkRows;
+        // exact rows: 64 (the last chunk fewer, known from the row count by then)
+        const int total = ctl[1];
+        const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * (k - kx0)) : kChunkRows;
         const int r16 = wg * 16;
         if (r16 < cnt) {
           float z[2][2];
@@ -880,6 +903,8 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
           ws.template update<true, kRows>(base + Gm::BOXB / 2, r16, lane, z, 1.f);
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * slot);   // the loaders may refill the slot
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -887,7 +912,6 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
 #pragma unroll
           for (int jj = 0; jj < 2; ++jj) sv[t][i][jj] = svn[t][i][jj];
     }
-    cp_wait_all();                           // this thread's gathers have landed (also on an error path)
   }
   // ---- combine ----
   cbar();                                  // every chunk is consumed: the ring is free

@@ -63,9 +63,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // Wait for the phase of `bar` with parity `parity`; gives up (false) once the
 // global timer passes `deadline` (ns).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long deadline) {
-  while (!mbar_try(bar, parity))
-    if (gtimer() > deadline) return false;
-  return true;
+  // the global timer is read once every 64 polls: a poll is cheap, a timer read is not
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 63u) == 0u && gtimer() > deadline) return false;
+  }
 }
 // one tile of a 2-D tensor map (columns x, rows y) into shared memory
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t bar) {

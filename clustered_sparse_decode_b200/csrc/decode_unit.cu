@@ -66,7 +66,7 @@ constexpr int kMinNS = 4;
 constexpr int kMaxSpt = 16;                    // selection: slots per compute thread
 constexpr int kMaxSlots = kMaxSpt * kCT;       // 4096
 constexpr int kMaxCluster = 8;
-constexpr int kFullCount = kLoaders * kWarp;   // arrivals completing a full slot: one per loader thread
+constexpr int kFullCount = kWarp;              // arrivals completing a full slot: one per lane of its loader
 constexpr int kSmemLimit = 232448;             // dynamic shared memory of one CTA per SM
 constexpr int kBarC = 2;                       // named barrier: compute threads
 
@@ -184,6 +184,15 @@ __device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
   return v;
 }
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync %0, %1;\n" ::"n"(kBarC), "n"(kCT) : "memory"); }
+// shared-memory acquire load / release store of a flag (CTA scope)
+__device__ __forceinline__ int ld_acquire(volatile int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(smem_u32(const_cast<int*>(p))) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(volatile int* p, int v) {
+  asm volatile("st.release.cta.shared.b32 [%0], %1;\n" ::"r"(smem_u32(const_cast<int*>(p))), "r"(v) : "memory");
+}
 // named barrier `id` of n threads
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
 
@@ -464,7 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
       volatile int* ctl = reinterpret_cast<volatile int*>(smem + a.o_q + kRowCap * 4);
       ctl[0] = 0;
       ctl[1] = -1;
-      for (int i = 0; i < kLoaders; ++i) ctl[2 + i] = 0;
+      for (int i = 0; i < kLoaders; ++i) ctl[2 + i] = 0x3fffffff;   // loaders that gather no exact chunk
+      ctl[2] = ctl[3] = 0;
+      if (NS % 3 == 0) ctl[4] = 0;   // a third loader gathers when the ring is a multiple of 3
       for (int i = 0; i < kMaxNS; ++i) ctl[8 + i] = -1;   // gen[]: no exact chunk's slot handed over yet
     }
   }
@@ -529,65 +540,40 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
     }
     if constexpr (MODE == M_FLAT) {
       if (li < kLoaders) {
-        // ---------------- exact chunks (loader li) ----------------
-        // A slot's empty barrier may be waited on only one phase ahead of its
-        // last completed phase (the parity test cannot tell phases two apart).
-        // Loaders 1..3 issue no tile chunk, so for the first NS exact chunks,
-        // whose slots last held tile chunks, they take loader 0's word that the
-        // slot is free (gen[slot] = the chunk loader 0 acquired it for).
+        // ---------------- exact chunks ----------------
+        // Exact chunk k is gathered whole by loader (k mod NS) mod nl: each slot
+        // always takes the same loader, which waits for the slot's releases one
+        // phase after the other (an empty barrier's parity test cannot tell
+        // phases two apart).  The first NS exact chunks' slots last held tile
+        // chunks: loader 0 follows those releases in order and hands each slot
+        // over (gen[slot] = the chunk it is free for).
+        const int nl = NS % 3 == 0 ? 3 : 2;    // loaders of exact chunks
         volatile int* gen = ctl + 8;
-#pragma unroll 1
-        for (int j = 0; ok; ++j) {
-          const int k = kx0 + j;
-          // the chunk's rows are published, or all rows are known (then possibly none left)
-          int total = -1, avail = 0;
+        // rows of exact chunk j: its count (0: past the rows; -1: timed out)
+        auto chunk_rows = [&](int j) -> int {
 #pragma unroll 1
           for (int spins = 0;; ++spins) {
-            total = __shfl_sync(kFull, ctl[1], 0);
-            avail = __shfl_sync(kFull, ctl[0], 0);
-            if (total >= 0 || avail >= kChunkRows * (j + 1)) break;
-            if ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline)) { ok = false; break; }
+            // acquire loads: the queue entries below the published count are visible after them
+            const int total = __shfl_sync(kFull, ld_acquire(&ctl[1]), 0);
+            const int avail = __shfl_sync(kFull, ld_acquire(&ctl[0]), 0);
+            if (total >= 0) return max(0, min(kChunkRows, total - kChunkRows * j));
+            if (avail >= kChunkRows * (j + 1)) return kChunkRows;
+            if ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline)) return -1;
             __nanosleep(64);
           }
-          if (!ok) {
-            if (lane == 0) set_error(a.err, E_TIMEOUT);
-            break;
-          }
-          __threadfence_block();               // the published rows, after their count
-          if (total >= 0 && kChunkRows * j >= total) break;
-          const int cnt = total >= 0 ? min(kChunkRows, total - kChunkRows * j) : kChunkRows;
-          const int i0 = 16 * li;
-          const int r = (lane < 16 && i0 + lane < cnt) ? rowq[(kChunkRows * j + i0 + lane) % kRowCap] : -1;
-          __threadfence_block();
-          __syncwarp();
-          if (lane == 0) ctl[2 + li] = j + 1;  // this loader has read its entries of chunk j
-          if (li == 0 || k >= kx0 + NS) {
-            ok = acquire(k);
-            if (li == 0 && k < kx0 + NS) {
-              __syncwarp();
-              if (lane == 0) gen[k % NS] = ok ? k : -2;
-            }
-          } else {
-#pragma unroll 1
-            for (int spins = 0;; ++spins) {
-              const int g = __shfl_sync(kFull, gen[k % NS], 0);
-              if (g == k) break;
-              if (g == -2 || ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline))) { ok = false; break; }
-              __nanosleep(32);
-            }
-            if (!ok && lane == 0) set_error(a.err, E_TIMEOUT);
-          }
-          if (!ok) break;
+        };
+        auto gather = [&](int k, int j, int cnt) {
+          const int r0 = lane < cnt ? rowq[(kChunkRows * j + lane) % kRowCap] : -1;
+          const int r1 = lane + 32 < cnt ? rowq[(kChunkRows * j + 32 + lane) % kRowCap] : -1;
           const uint32_t dst = sb + (k % NS) * Gm::SLOT;
           if constexpr (D == 128) {
             // one row (keys and values, 2 x 256 B) per instruction: lane = kv:1 half:1 c16:3
             const int kv = lane >> 4, half = (lane >> 3) & 1, c16 = lane & 7;
             const char* g = (kv ? a.Vp : a.Kp) + half * 128 + c16 * 16;
             const uint32_t d0 = dst + kv * (Gm::BOXB / 2) + half * (Gm::BOXB / 4);
-#pragma unroll
-            for (int s2 = 0; s2 < 16; ++s2) {
-              const int rw = __shfl_sync(kFull, r, s2);
-              const int i = i0 + s2, rr = i & 7;
+#pragma unroll 8
+            for (int i = 0; i < kChunkRows; ++i) {
+              const int rw = __shfl_sync(kFull, i < 32 ? r0 : r1, i & 31), rr = i & 7;
               cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)max(rw, 0) * 256, rw >= 0);
             }
           } else {
@@ -595,14 +581,57 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
             const int sub = lane >> 4, kv = (lane >> 3) & 1, c16 = lane & 7;
             const char* g = (kv ? a.Vp : a.Kp) + c16 * 16;
             const uint32_t d0 = dst + kv * (Gm::BOXB / 2);
-#pragma unroll
-            for (int s2 = 0; s2 < 16; s2 += 2) {
-              const int rw = __shfl_sync(kFull, r, s2 + sub);
-              const int i = i0 + s2 + sub, rr = i & 7;
+#pragma unroll 8
+            for (int i2 = 0; i2 < kChunkRows; i2 += 2) {
+              const int i = i2 + sub;
+              const int rw = __shfl_sync(kFull, i2 < 32 ? r0 : r1, i & 31), rr = i & 7;
               cp16(d0 + (i >> 3) * Gm::BOXB + rr * 128 + ((c16 ^ rr) << 4), g + (size_t)max(rw, 0) * 128, rw >= 0);
             }
           }
-          cp_arrive_noinc(full0 + 8 * (k % NS));   // one of the slot's 128 arrivals, once this lane's copies land
+          cp_arrive_noinc(full0 + 8 * (k % NS));   // one of the slot's 32 arrivals, once this lane's copies land
+          // every copy above consumed its entry: the planner may reuse the chunk's entries
+          __syncwarp();
+          if (lane == 0) ctl[2 + li] = j + 1;
+        };
+        if (li < nl) {
+          // loader 0: hand over the first NS exact slots, gathering its own among them
+          if (li == 0) {
+#pragma unroll 1
+            for (int k = kx0; k < kx0 + NS && ok; ++k) {
+              ok = acquire(k);
+              __syncwarp();
+              if (lane == 0) gen[k % NS] = ok ? k : -2;
+              if (!ok || (k % NS) % nl != 0) continue;
+              const int cnt = chunk_rows(k - kx0);
+              if (cnt < 0) { ok = false; if (lane == 0) set_error(a.err, E_TIMEOUT); break; }
+              if (cnt == 0) break;
+              gather(k, k - kx0, cnt);
+            }
+          }
+          // then every chunk of this loader's slots, in order
+          const int k_first = li == 0 ? kx0 + NS : kx0;
+#pragma unroll 1
+          for (int k = k_first; ok; ++k) {
+            if ((k % NS) % nl != li) continue;
+            const int j = k - kx0;
+            const int cnt = chunk_rows(j);
+            if (cnt < 0) { ok = false; if (lane == 0) set_error(a.err, E_TIMEOUT); break; }
+            if (cnt == 0) break;
+            if (k >= kx0 + NS) {
+              ok = acquire(k);
+            } else {
+#pragma unroll 1
+              for (int spins = 0;; ++spins) {
+                const int g = __shfl_sync(kFull, gen[k % NS], 0);
+                if (g == k) break;
+                if (g == -2 || ((spins & 63) == 63 && __any_sync(kFull, gtimer() > deadline))) { ok = false; break; }
+                __nanosleep(32);
+              }
+              if (!ok && lane == 0) set_error(a.err, E_TIMEOUT);
+            }
+            if (!ok) break;
+            gather(k, j, cnt);
+          }
         }
         cp_wait_all();                         // this warp's copies have landed (also on an error path)
       } else {
@@ -703,15 +732,13 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
             const int before = __shfl_sync(kFull, incl - cnt, lo);
             const int rs = __shfl_sync(kFull, st, lo);
             if (q < nrows) rowq[(written + q) % kRowCap] = unit_row + rs + (q - before);
-            __threadfence_block();
             __syncwarp();
-            if (lane == 0) ctl[0] = written + min(b0 + 32, nrows);
+            if (lane == 0) st_release(&ctl[0], written + min(b0 + 32, nrows));
           }
           written += nrows;
         }
-        __threadfence_block();
         __syncwarp();
-        if (lane == 0) ctl[1] = ok ? written : 0;
+        if (lane == 0) st_release(&ctl[1], ok ? written : 0);
       }
     }
     if (K > 1) {

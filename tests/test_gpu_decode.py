@@ -161,7 +161,7 @@ def test_selection_with_exact_score_ties(budget, dtype):
     """The selection as a function of the scores it reports: groups of 64 and of
     4 clusters with identical keys (exact score ties at the crossing, more and
     fewer candidates than one warp resolves) and one unit of distinct keys;
-    bf16 runs the two-pass kernels, fp32 the multi-kernel path."""
+    bf16 runs the one-kernel unit decode, fp32 the multi-kernel path."""
     o = H.ocfg(B=1, Hkv=3, Hq=12, d=128, n_max=4096, T=16, L_blk=4096, dtype=dtype)
     rng = np.random.default_rng(12)
     K = np.empty((1, 3, 4096, 128), dtype=np.float32)
@@ -272,9 +272,9 @@ def test_full_size_bench_launch_sampled_units():
 @pytest.mark.parametrize("n", [0, 5, 8, 500])
 def test_unclustered_indices(n):
     """Indices holding only a tail (appended tokens below the update interval):
-    empty (O = 0), fewer than 8 tokens (the multi-kernel path), exactly 8 and
-    500 tokens (the two-pass path with no clusters).  Every token is attended
-    exactly: the oracle's decode of its own appended index."""
+    empty (O = 0), 5, 8 and 500 tokens (a tail only, no cluster: the unit
+    decode's exact stream alone, a partial chunk for 5 and 8).  Every token is
+    attended exactly: the oracle's decode of its own appended index."""
     o = H.ocfg(B=2, Hkv=2, Hq=8, d=128, n_max=4096, T=16, L_blk=2048, update_interval=1024)
     K, V, _ = H.cache_for(o, max(n, 1), comps=8, seed=30 + n)
     oidx = mp.empty_index(o)

@@ -432,6 +432,223 @@ __device__ void select_smem(const Args& a, const float* shat, const int32_t* off
   }
 }
 
+// The same selection with the slots held in registers: thread t owns the SPT
+// consecutive slots [SPT t, SPT t + SPT) (16-byte loads of the group scores
+// and offsets, once), and every pass works on those registers, so a pass costs
+// a few instructions per slot instead of dependent shared-memory loads.  The
+// selection bits of 32 slots are assembled from the owning threads' bits with
+// shuffles.  SPT = 8 covers 2048 slots, 16 covers 4096.
+template <int SPT>
+__device__ void select_vec(const Args& a, const float* shat, const int32_t* offs, uint32_t* selm, int* red,
+                           int* hist, int u, bool write_out) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slots = a.rows_active;
+  const int c0 = tid * SPT;
+  uint32_t key[SPT];
+  int w[SPT];
+  {
+    float sc[SPT];
+    int of[SPT + 1];
+    if (c0 + SPT <= slots) {
+#pragma unroll
+      for (int i = 0; i < SPT / 4; ++i) {
+        const float4 s4 = reinterpret_cast<const float4*>(shat + c0)[i];
+        const int4 o4 = reinterpret_cast<const int4*>(offs + c0)[i];
+        sc[4 * i] = s4.x; sc[4 * i + 1] = s4.y; sc[4 * i + 2] = s4.z; sc[4 * i + 3] = s4.w;
+        of[4 * i] = o4.x; of[4 * i + 1] = o4.y; of[4 * i + 2] = o4.z; of[4 * i + 3] = o4.w;
+      }
+      of[SPT] = offs[c0 + SPT];
+    } else {
+#pragma unroll
+      for (int i = 0; i < SPT; ++i) {
+        sc[i] = c0 + i < slots ? shat[c0 + i] : 0.f;
+        of[i] = c0 + i <= slots ? offs[c0 + i] : 0;
+      }
+      of[SPT] = c0 + SPT <= slots ? offs[c0 + SPT] : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < SPT; ++i) {
+      const int cnt = c0 + i < slots ? of[i + 1] - of[i] : 0;
+      w[i] = cnt > 0 ? cnt : 0;
+      key[i] = cnt > 0 ? ordered_key(sc[i]) : 0u;
+    }
+  }
+  // 1. total weight, smallest and largest key of the non-empty clusters
+  int wsum = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < SPT; ++i)
+    if (w[i] > 0) {
+      wsum += w[i];
+      kmin = min(kmin, key[i]);
+      kmax = max(kmax, key[i]);
+    }
+  {
+    const int ws_ = __reduce_add_sync(kFull, wsum);
+    const uint32_t mn = __reduce_min_sync(kFull, kmin), mx = __reduce_max_sync(kFull, kmax);
+    if (lane == 0) { red[warp] = ws_; red[kCW + warp] = (int)mn; red[2 * kCW + warp] = (int)mx; }
+    cbar();
+    wsum = 0; kmin = 0xffffffffu; kmax = 0u;
+#pragma unroll
+    for (int i = 0; i < kCW; ++i) {
+      wsum += red[i];
+      kmin = min(kmin, (uint32_t)red[kCW + i]);
+      kmax = max(kmax, (uint32_t)red[2 * kCW + i]);
+    }
+    cbar();
+  }
+  const int W = wsum;
+  const int mode = (a.budget <= 0 || W == 0) ? 0 : (W <= a.budget ? 1 : 2);   // none | all | threshold
+  uint32_t tau = 0u;
+  int ntie = 0, above = 0;
+  bool resolved = false;
+  if (mode == 2) {
+    // 2a. 256 equal-width score bins; the crossing bin's clusters, if at most 32, ranked by one warp
+    const float smin = key_score(kmin), smax = key_score(kmax);
+    const float span = smax - smin, inv = 256.f / span;
+    if (isfinite(smin) && isfinite(smax) && span > 0.f && isfinite(span) && isfinite(inv)) {
+      auto fbin = [&](uint32_t kk) { return min(255, (int)((key_score(kk) - smin) * inv)); };
+      int* lst = hist + 256;                                // [32][3] candidates of the crossing bin
+      for (int i = tid; i < 256; i += kCT) hist[i] = 0;
+      if (tid == 0) red[3] = 0;
+      cbar();
+#pragma unroll
+      for (int i = 0; i < SPT; ++i)
+        if (w[i] > 0) atomicAdd(hist + fbin(key[i]), w[i]);
+      cbar();
+      if (warp == 0) crossing_bin(hist, 0, a.budget, lane, red);
+      cbar();
+      const int fb = red[0], ab = red[1];
+#pragma unroll
+      for (int i = 0; i < SPT; ++i)
+        if (w[i] > 0 && fbin(key[i]) == fb) {
+          const int pos = atomicAdd(red + 3, 1);
+          if (pos < 32) { lst[3 * pos] = (int)key[i]; lst[3 * pos + 1] = c0 + i; lst[3 * pos + 2] = w[i]; }
+        }
+      cbar();
+      const int nc = red[3];
+      if (nc <= 32) {
+        if (warp == 0) {
+          // lane l holds candidate l (key, weight); the crossing key t is the
+          // largest key whose candidates at or above it bring the running
+          // weight ab + W(key >= t) to the budget
+          const uint32_t kl = lane < nc ? (uint32_t)lst[3 * lane] : 0u;
+          const int wl = lane < nc ? lst[3 * lane + 2] : 0;
+          int wgt = 0, weq = 0;
+#pragma unroll 1
+          for (int j = 0; j < nc; ++j) {
+            const uint32_t kj = (uint32_t)__shfl_sync(kFull, (int)kl, j);
+            const int wj = __shfl_sync(kFull, wl, j);
+            wgt += kj > kl ? wj : 0;
+            weq += kj == kl ? wj : 0;
+          }
+          const bool reach = lane < nc && ab + wgt + weq >= a.budget;
+          const uint32_t t = __reduce_max_sync(kFull, reach ? kl : 0u);
+          const int tl = __ffs(__ballot_sync(kFull, reach && kl == t)) - 1;
+          const int gt = __shfl_sync(kFull, wgt, tl);
+          const int nt = __popc(__ballot_sync(kFull, lane < nc && kl == t));
+          if (lane == 0) { red[0] = (int)t; red[1] = ab + gt; red[2] = nt; }
+        }
+        cbar();
+        tau = (uint32_t)red[0];
+        above = red[1];
+        ntie = red[2];
+        resolved = true;
+      }
+      cbar();
+    }
+  }
+  if (mode == 2 && !resolved) {
+    // 2b. radix descent over the keys in [kmin, kmax], 8 bits at a time
+    uint32_t lo = kmin;
+    int nb = kmax == kmin ? 0 : 32 - __clz(kmax - kmin);
+    above = 0;
+    int* hcnt = hist + 256;
+    ntie = -1;
+#pragma unroll 1
+    while (nb > 0) {
+      const int sh = max(nb - 8, 0);
+      for (int i = tid; i < 256; i += kCT) { hist[i] = 0; hcnt[i] = 0; }
+      cbar();
+      const unsigned long long hi_excl = (unsigned long long)lo + (1ull << nb);
+#pragma unroll
+      for (int i = 0; i < SPT; ++i)
+        if (w[i] > 0 && key[i] >= lo && (unsigned long long)key[i] < hi_excl) {
+          const int bin = (int)((key[i] - lo) >> sh);
+          atomicAdd(hist + bin, w[i]);
+          if (sh == 0) atomicAdd(hcnt + bin, 1);
+        }
+      cbar();
+      if (warp == 0) {
+        crossing_bin(hist, above, a.budget, lane, red);
+        __syncwarp();
+        if (lane == 0) red[2] = hcnt[red[0]];
+      }
+      cbar();
+      const int bsel = red[0];
+      above = red[1];
+      if (sh == 0) ntie = red[2];
+      lo += (uint32_t)bsel << sh;
+      nb = sh;
+      cbar();
+    }
+    tau = lo;
+  }
+  // 3. the selection bits: every cluster above tau, and the one at tau when
+  // no other cluster ties with it (it is the crossing cluster: always taken)
+  {
+    uint32_t mine = 0u;
+#pragma unroll
+    for (int i = 0; i < SPT; ++i) {
+      bool sel = false;
+      if (w[i] > 0) sel = mode == 1 || (mode == 2 && (key[i] > tau || (ntie == 1 && key[i] == tau)));
+      mine |= sel ? (1u << i) : 0u;
+    }
+    constexpr int TPW = 32 / SPT;                        // threads per 32-slot word
+    uint32_t word = mine << (SPT * (tid % TPW));
+#pragma unroll
+    for (int o = 1; o < TPW; o <<= 1) word |= __shfl_xor_sync(kFull, word, o);
+    if (tid % TPW == 0 && c0 < slots) selm[c0 >> 5] = word;
+  }
+  cbar();
+  if (mode == 2 && ntie != 1) {
+    // several clusters exactly at tau: taken in slot order while the tokens
+    // taken among them stay below budget - above (one warp; ties are rare)
+    if (warp == 0) {
+      const int need = a.budget - above;
+      int taken = 0;
+#pragma unroll 1
+      for (int base = 0; base < slots && taken < need; base += 32) {
+        const int c = base + lane;
+        int tw = 0;
+        if (c < slots) {
+          const int ww = offs[c + 1] - offs[c];
+          if (ww > 0 && ordered_key(shat[c]) == tau) tw = ww;
+        }
+        int inc = tw;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const unsigned bits = __ballot_sync(kFull, tw > 0 && taken + inc - tw < need);
+        if (lane == 0 && bits) selm[base >> 5] |= bits;
+        taken += __shfl_sync(kFull, inc, 31);
+      }
+    }
+    cbar();
+  }
+  if (write_out) {
+#pragma unroll 1
+    for (int c = tid; c < a.rows; c += kCT) {
+      const bool in = c < slots && offs[c + 1] > offs[c];
+      const bool sel = c < slots && ((selm[c >> 5] >> (c & 31)) & 1u);
+      if (a.sel_mask_out) a.sel_mask_out[(size_t)u * a.rows + c] = sel ? 1 : 0;
+      if (a.scores_out) a.scores_out[(size_t)u * a.rows + c] = in ? shat[c] : -INFINITY;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
@@ -833,7 +1050,8 @@ __global__ void __launch_bounds__(kThreads, 1) unit_decode(const __grid_constant
       }
       cbar();
     }
-    select_smem<G>(a, shat, offs, selm, red, red + 256, u, rank == 0);
+    if (a.rows_active <= 8 * kCT) select_vec<8>(a, shat, offs, selm, red, red + 256, u, rank == 0);
+    else select_smem<G>(a, shat, offs, selm, red, red + 256, u, rank == 0);
     cbar();                                // every read of the group scores is done
     if (threadIdx.x == 0) mbar_arrive(selready);   // the loaders may pack the selected rows (over the group scores)
   }

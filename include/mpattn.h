@@ -225,11 +225,12 @@ mp_status mp_decode(const mp_index* idx, const void* Q, void* O, const mp_decode
  * loads the library holds until the process exits.  It calls no allocator.
  *  - Returns MP_ENOSPC if the configuration's decode_scratch_bytes
  *    (mp_workspace_size) exceed MP_STATIC_SCRATCH_BYTES.
- *    A flat bf16 index needs only room for a staged Q (B * Hq * d * 2
- *    bytes: 128 KiB at batch 16, 32 query heads, d 128), so every flat bf16
- *    configuration up to 4096 query rows of d 128 fits; fp32 and two-level
- *    indexes need the multi-kernel path's partials and run lists, which grow
- *    with batch x heads x slots.
+ *    A flat bf16 index needs the per-head centroid scores (B * Hkv * slots *
+ *    4 * ceil(G / 4) * 4 bytes: 4 MiB at batch 16, 8 KV heads, 2048 slots,
+ *    G = 4) plus room for a staged Q (B * Hq * d * 2 bytes: 128 KiB there),
+ *    so flat bf16 configurations up to about 8 times that shape fit; fp32 and
+ *    two-level indexes need the multi-kernel path's partials and run lists,
+ *    which grow with batch x heads x slots.
  *  - The first call on each device, and the first after the device's current
  *    context changed (cudaDeviceReset, another driver-API context made
  *    current), looks up the array's device address (cudaGetSymbolAddress)

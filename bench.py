@@ -771,6 +771,96 @@ def source_digest(kernel=None):
     return h.hexdigest()[:12]
 
 
+SWEEP_T = (8, 16, 32, 64, 128)
+SWEEP_BLOCK = (2048, 4096, 8192, 16384)
+
+
+def run_sweep(args):
+    """The ablation knobs of the pages as a speed sweep (NEXT-2): tokens per centroid T x
+    clustering block size, on one seeded batch-4, 32K-token cache (the bench's key and value
+    distribution) with the bench's 5% budget.  Each configuration builds its own index (timed)
+    and decodes `steps` queries with the L2 flushed before each (CUDA events).  Prints one JSON
+    line; with --sweep-out also writes the table as markdown."""
+    import torch
+    from clustered_sparse_decode_b200 import Config, MultipoleIndex, synth
+    from clustered_sparse_decode_b200 import build as libbuild
+    libbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    base = synth.workload("batch4_32k_sparse95")
+    B, Hkv, Hq, d, n = base["B"], base["Hkv"], base["Hq"], base["d"], base["n"]
+    K, V, _ = synth.make_cache(B, Hkv, n, d, base["comps"], base["sigma"], radius=base["radius"],
+                               outliers=base["outliers"], dtype="bf16", seed=base["seed"])
+    Kd = torch.from_numpy(K).to(dev).to(torch.bfloat16)
+    Vd = torch.from_numpy(V).to(dev).to(torch.bfloat16)
+    del K, V
+    steps = min(args.steps, 20)
+    Q = torch.from_numpy(synth.make_queries(args.warmup + steps, B, Hq, d, "bf16", seed=base["seed"] + 7)) \
+        .to(dev).to(torch.bfloat16)
+    O = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    pk = peaks()
+    flush = make_flusher(dev)
+    budget = base["budget"]
+    clocks = ClockSampler(0)
+    clocks.start()
+    rows = []
+    for T in SWEEP_T:
+        for L in SWEEP_BLOCK:
+            w = dict(base, T=T, L_blk=L)
+            cfg = Config(batch=B, kv_heads=Hkv, q_heads=Hq, head_dim=d, max_tokens=n, tokens_per_centroid=T,
+                         block_tokens=L, kmeans_iters=base["iters"], dtype="bf16", seed=base["seed"])
+            idx = MultipoleIndex(cfg, device=dev)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            idx.build(Kd, Vd)
+            torch.cuda.synchronize()
+            build_s = time.perf_counter() - t0
+            if idx.check_device_error() != 0:
+                raise RuntimeError(f"device error after the T={T}, block={L} build")
+            # algorithmic bytes from each timed step's own selection (untimed pass)
+            off = idx.arrays()["off"].to(torch.int64)
+            cnt = off[:, :, 1:] - off[:, :, :-1]
+            C_unit = (cnt > 0).sum(dim=2)
+            mask = torch.zeros((B, Hkv, idx.slots), dtype=torch.uint8, device=dev)
+            step_bytes, sel_tokens = [], []
+            for i in range(args.warmup, args.warmup + steps):
+                idx.decode(Q[i], budget, out=O, sel_mask=mask)
+                nsel = (cnt * mask.to(torch.int64)).sum(dim=2)
+                sel_tokens.append(float(nsel.to(torch.float64).mean()))
+                step_bytes.append(sum(algorithmic_bytes_unit(w, int(C_unit[b, h]), int(nsel[b, h]), 0)
+                                      for b in range(B) for h in range(Hkv)))
+            ms = time_steps(lambda i: idx.decode(Q[i], budget, out=O), steps, args.warmup, flush)
+            if idx.check_device_error() != 0:
+                raise RuntimeError(f"device error in the T={T}, block={L} decode")
+            us = 1e3 * statistics.mean(ms)
+            gbs = sum(step_bytes) / (sum(ms) / 1e3) / 1e9
+            rows.append({"T": T, "block_tokens": L, "slots_per_head": idx.slots, "us_per_step": us, "gb_s": gbs,
+                         "frac_hbm": gbs / pk["hbm_gbs"], "bytes_per_step": statistics.mean(step_bytes),
+                         "selected_tokens_per_head": statistics.mean(sel_tokens), "build_s": build_s})
+            del idx
+            torch.cuda.empty_cache()
+    clk = clocks.stop()
+    head = next(r for r in rows if r["T"] == 16 and r["block_tokens"] == 8192)
+    line = {"metric": "decode µs/step and build s per (tokens per centroid, block size), B=4, 32K ctx, 5% budget",
+            "value": head["gb_s"], "unit": "GB/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": head["us_per_step"] / 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "sweep (batch4_32k_sparse95 cache; T x block)", "batch": B, "kv_heads": Hkv,
+                       "q_heads": Hq, "head_dim": d, "context": n, "budget": budget,
+                       "l2": "flushed between timed steps (2x L2 written, then 2x L2 read: cold and clean)"},
+            "clocks": clk, "sweep": rows}
+    print(json.dumps(line), flush=True)
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            f.write("| T (tokens per centroid) | block tokens | slots per head | µs/step | GB/s | % of HBM | "
+                    "selected tokens per head | build s |\n|---|---|---|---|---|---|---|---|\n")
+            for r in rows:
+                f.write(f"| {r['T']} | {r['block_tokens']} | {r['slots_per_head']} | {r['us_per_step']:.1f} | "
+                        f"{r['gb_s']:.0f} | {100 * r['frac_hbm']:.1f}% | {r['selected_tokens_per_head']:.0f} | "
+                        f"{r['build_s']:.3f} |\n")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -786,9 +876,14 @@ def main(argv=None):
                     help="skip the other configurations (dense baseline, single sequence, two-level, online)")
     ap.add_argument("--gen-tokens", type=int, default=0,
                     help="online workloads: generated tokens to time (0 = all of the workload's)")
+    ap.add_argument("--sweep-out", default=None, help="--workload sweep: also write the table as markdown here")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "sweep":
+        if args.impl == "reference" or args.gpus != 1:
+            ap.error("--workload sweep runs our implementation on one GPU")
+        return run_sweep(args)
     from clustered_sparse_decode_b200 import synth
     w = synth.workload(args.workload)
     if args.impl == "reference":

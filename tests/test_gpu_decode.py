@@ -129,12 +129,14 @@ def test_hierarchical_decode_matches_oracle(coarse_budget, budget, no_approx):
     run_decode(o, oidx, Q, budget, coarse_budget=coarse_budget, no_approx=no_approx)
 
 
-@pytest.mark.parametrize("levels", [1, 2])
-def test_4096_slot_units_decode(levels):
-    """One unit of 64K tokens at 16 tokens per centroid: 4096 slots, whose
-    selection keys fill the 48 KB default shared-memory window exactly (fp32
-    flat index on the multi-kernel path, and the hierarchical index)."""
-    dt = "f32" if levels == 1 else "bf16"
+@pytest.mark.parametrize("levels,dt", [(1, "f32"), (2, "bf16"), (1, "bf16")])
+def test_4096_slot_units_decode(levels, dt):
+    """One unit of 64K tokens at 16 tokens per centroid: 4096 slots.  The fp32
+    flat index runs the multi-kernel path (its selection keys fill the 48 KB
+    default shared-memory window exactly), the hierarchical index the
+    two-level path, and the bf16 flat index the one-kernel decode with its
+    largest unit (a ring of 4 slots, the shared-memory selection for more
+    than 2048 slots)."""
     o = H.ocfg(B=1, Hkv=1, Hq=4, d=128, n_max=65536, T=16, L_blk=8192, levels=levels, Tc=128, dtype=dt)
     K, V, lab = H.cache_for(o, 65536, comps=512, seed=21)
     oidx = H.component_index(o, K, V, lab, 65536)

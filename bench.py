@@ -777,8 +777,8 @@ SWEEP_BLOCK = (2048, 4096, 8192, 16384)
 
 def run_sweep(args):
     """The ablation knobs of the pages as a speed sweep (NEXT-2): tokens per centroid T x
-    clustering block size, on one seeded batch-4, 32K-token cache (the bench's key and value
-    distribution) with the bench's 5% budget.  Each configuration builds its own index (timed)
+    clustering block size, on one seeded batch-4 (or, with --sweep-batch 16, the bench's batch-16)
+    32K-token cache (the bench's key and value distribution) with the bench's 5% budget.  Each configuration builds its own index (timed)
     and decodes `steps` queries with the L2 flushed before each (CUDA events).  Prints one JSON
     line; with --sweep-out also writes the table as markdown."""
     import torch
@@ -787,7 +787,7 @@ def run_sweep(args):
     libbuild.build()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(0)
-    base = synth.workload("batch4_32k_sparse95")
+    base = synth.workload("batch4_32k_sparse95" if args.sweep_batch == 4 else "batch16_32k_sparse95")
     B, Hkv, Hq, d, n = base["B"], base["Hkv"], base["Hq"], base["d"], base["n"]
     K, V, _ = synth.make_cache(B, Hkv, n, d, base["comps"], base["sigma"], radius=base["radius"],
                                outliers=base["outliers"], dtype="bf16", seed=base["seed"])
@@ -841,11 +841,11 @@ def run_sweep(args):
             torch.cuda.empty_cache()
     clk = clocks.stop()
     head = next(r for r in rows if r["T"] == 16 and r["block_tokens"] == 8192)
-    line = {"metric": "decode µs/step and build s per (tokens per centroid, block size), B=4, 32K ctx, 5% budget",
+    line = {"metric": f"decode µs/step and build s per (tokens per centroid, block size), B={B}, 32K ctx, 5% budget",
             "value": head["gb_s"], "unit": "GB/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
             "ms_per_step": head["us_per_step"] / 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "sweep (batch4_32k_sparse95 cache; T x block)", "batch": B, "kv_heads": Hkv,
+            "config": {"workload": f"sweep (batch{B}_32k_sparse95 cache; T x block)", "batch": B, "kv_heads": Hkv,
                        "q_heads": Hq, "head_dim": d, "context": n, "budget": budget,
                        "l2": "flushed between timed steps (2x L2 written, then 2x L2 read: cold and clean)"},
             "clocks": clk, "sweep": rows}
@@ -877,6 +877,8 @@ def main(argv=None):
     ap.add_argument("--gen-tokens", type=int, default=0,
                     help="online workloads: generated tokens to time (0 = all of the workload's)")
     ap.add_argument("--sweep-out", default=None, help="--workload sweep: also write the table as markdown here")
+    ap.add_argument("--sweep-batch", type=int, choices=[4, 16], default=4,
+                    help="--workload sweep: the cache's batch (4, or 16 = the bench geometry)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

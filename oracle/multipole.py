@@ -606,7 +606,7 @@ def _scores(q, cents, scale):
 
 
 def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, force_sel=None,
-           units=None):
+           units=None, per_head=False):
     """One decode step for every (batch, query head).  Returns O [B, Hq, d] (fp64).
 
     Flat index (levels == 1), per KV head h and its query heads g (R1):
@@ -627,6 +627,13 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, f
     than one set be correct, this gives the output that belongs to a particular
     one of them.  ``units`` (optional): the (b, h) pairs to compute; the output
     rows of the other units are left zero.
+
+    ``per_head`` (flat index only): the other reading of R1 left open by the
+    pages — every query head g selects on its own scores S[g, c] instead of the
+    group max, with the same token budget, and its softmax takes exact terms
+    for its own selected clusters (and the tail) and centroid terms for its own
+    unselected clusters.  A KV head then reads the union of its query heads'
+    selections.  ``info`` receives the per-head sets as ``sel_heads``.
     """
     cfg = idx["cfg"]
     B, H, Hq, d = cfg["B"], cfg["Hkv"], cfg["Hq"], cfg["d"]
@@ -636,6 +643,8 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, f
     if coarse_budget is None:
         coarse_budget = 8 * budget
     nc, nt = idx["n_clustered"], idx["n_tokens"]
+    if per_head and (cfg.get("levels", 1) != 1 or force_sel is not None):
+        raise ValueError("per_head selection is defined for flat indices without forced sets")
     O = np.zeros((B, Hq, d))
     todo = None if units is None else {tuple(u) for u in units}
     for b in range(B):
@@ -651,6 +660,23 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, f
             S = _scores(q, Kc, scale)
             shat = np.where(cnt > 0, S.max(axis=0), -np.inf)
             unit_info = {}
+            if per_head:
+                sel_heads = []
+                for gi in range(G):
+                    sel_g, _ = select_clusters(np.where(cnt > 0, S[gi], -np.inf), cnt, budget)
+                    approx_g = np.setdiff1d(np.nonzero(cnt > 0)[0], sel_g)
+                    tok = [np.arange(off[c], off[c + 1]) for c in sel_g] + [np.arange(nc, nt)]
+                    tok = np.concatenate(tok).astype(np.int64)
+                    z = [scale * (Kp[tok] @ q[gi])]
+                    vals = [Vp[tok]]
+                    if not (flags & NO_APPROX):
+                        z.append(S[gi, approx_g] + np.log(cnt[approx_g]))
+                        vals.append(Vc[approx_g])
+                    O[b, h * G + gi] = _softmax_terms(np.concatenate(z), np.concatenate(vals, axis=0))
+                    sel_heads.append(sel_g)
+                if info is not None:
+                    info[(b, h)] = {"sel_heads": sel_heads, "S": S}
+                continue
             if cfg.get("levels", 1) == 1:
                 sel, ranked = select_clusters(shat, cnt, budget)
                 if forced is not None:

@@ -516,3 +516,76 @@ def test_forcing_every_cluster_is_dense_and_forcing_none_is_all_centroids():
         z = (Kc @ Q[0, g]) / math.sqrt(cfg["d"]) + np.log(cnt[nz])
         p = np.exp(z - z.max())
         np.testing.assert_allclose(O_none[0, g], p @ Vc / p.sum(), atol=1e-12)
+
+
+# --------------------------------------------------------------------------- per-query-head selection (NEXT-3)
+
+def test_per_head_selection_equals_brute_force_on_tiny_index():
+    """Each query head selects on its own scores (the other reading of R1):
+    brute-force selection per head and the brute-force softmax of that head."""
+    cfg = ocfg(B=1, Hkv=1, Hq=3, d=6, n_max=40, T=4, L_blk=40)
+    K, V, _ = cache(cfg, 40, comps=3)
+    idx = mp.build_index(K, V, 40, cfg)
+    Q = synth.make_queries(1, 1, 3, 6, "f32", seed=9)[0]
+    scale = 1 / math.sqrt(6)
+    off = idx["off"][0, 0]
+    clusters = []
+    for c in range(len(off) - 1):
+        rows = range(off[c], off[c + 1])
+        clusters.append(([idx["Kp"][0, 0, r].tolist() for r in rows], [idx["Vp"][0, 0, r].tolist() for r in rows],
+                         idx["Kc"][0, 0, c].tolist(), idx["Vc"][0, 0, c].tolist()))
+    counts = [len(c[0]) for c in clusters]
+    differs = False
+    for budget in [1, 6, 13, 40]:
+        O = mp.decode(idx, Q, budget, per_head=True)
+        sels = []
+        for g in range(3):
+            S = [scale * math.fsum(a * b for a, b in zip(Q[0, g], cl[2])) for cl in clusters]
+            sel = brute.select(S, counts, budget)
+            sels.append(set(sel))
+            want = brute.decode_one(Q[0, g].tolist(), scale, clusters, set(sel))
+            np.testing.assert_allclose(O[0, g], want, atol=1e-12)
+        differs |= len({frozenset(x) for x in sels}) > 1
+    assert differs                    # the heads do select differently here
+
+
+def test_per_head_selection_with_one_query_head_is_the_group_selection():
+    cfg = ocfg(B=2, Hkv=2, Hq=2, n_max=256, L_blk=64, T=4)
+    K, V, _ = cache(cfg, 256)
+    idx = mp.build_index(K, V, 256, cfg)
+    Q = synth.make_queries(1, 2, 2, cfg["d"], "f32", seed=4)[0]
+    for budget in [0, 1, 30, 300]:
+        np.testing.assert_array_equal(mp.decode(idx, Q, budget, per_head=True), mp.decode(idx, Q, budget))
+
+
+def test_per_head_selection_with_identical_heads_is_the_group_selection():
+    cfg = ocfg(B=1, Hkv=2, Hq=8, n_max=256, L_blk=64, T=4)
+    K, V, _ = cache(cfg, 256, seed=2)
+    idx = mp.build_index(K, V, 256, cfg)
+    q = synth.make_queries(1, 1, 2, cfg["d"], "f32", seed=6)[0]
+    Q = np.repeat(q, 4, axis=1)                     # the 4 query heads of each KV head are equal
+    for budget in [1, 30, 100]:
+        np.testing.assert_allclose(mp.decode(idx, Q, budget, per_head=True), mp.decode(idx, Q, budget), atol=1e-13)
+
+
+def test_per_head_output_depends_on_its_own_query_only():
+    """Changing the other query heads of the group leaves a head's output
+    unchanged under per-head selection; under the group max it does not."""
+    cfg = ocfg(B=1, Hkv=1, Hq=4, n_max=256, L_blk=64, T=4)
+    K, V, _ = cache(cfg, 256, seed=3)
+    idx = mp.build_index(K, V, 256, cfg)
+    Q = synth.make_queries(2, 1, 4, cfg["d"], "f32", seed=8)
+    Q2 = Q[0].copy()
+    Q2[0, 1:] = Q[1][0, 1:] * 3.0                    # heads 1..3 replaced, head 0 kept
+    a = mp.decode(idx, Q[0], 20, per_head=True)
+    b = mp.decode(idx, Q2, 20, per_head=True)
+    np.testing.assert_array_equal(a[0, 0], b[0, 0])
+    assert not np.array_equal(mp.decode(idx, Q[0], 20)[0, 0], mp.decode(idx, Q2, 20)[0, 0])
+
+
+def test_per_head_selection_with_the_whole_budget_is_dense_attention():
+    cfg = ocfg(B=1, Hkv=2, Hq=4, n_max=256, L_blk=64, T=4)
+    K, V, _ = cache(cfg, 200, seed=1)
+    idx = mp.build_index(K, V, 200, cfg)
+    Q = synth.make_queries(1, 1, 4, cfg["d"], "f32", seed=2)[0]
+    np.testing.assert_allclose(mp.decode(idx, Q, 10 ** 6, per_head=True), sdpa(Q, K, V, 200, 2), atol=1e-12)

@@ -5,7 +5,9 @@ Workload (default): batch 16, 8 KV / 32 query heads, head_dim 128, 32768 cached
 tokens per sequence, token budget 1638 (5% of the context, "95% sparsity"),
 seeded Gaussian-mixture keys (1 centroid per 16 tokens, 8K-token clustering
 blocks), bf16.  One step = one decode step of one attention layer for the
-whole batch (centroid pass, selection, token pass, combine).
+whole batch: one kernel launch on the bf16 path (centroid scores, selection,
+centroid terms, exact rows, combine), four on the multi-kernel path (fp32 and
+two-level indexes: centroid pass, selection, token pass, combine).
 
 Reports algorithmic HBM GB/s (the bytes the method must read: all key and value
 centroids, the run offsets, the selected clusters' keys and values, the

@@ -361,6 +361,101 @@ def _coarse_block(idx, b, h, j, L, tok0, unit):
     return {"coarse_assign": ca, "fine_order": fo, "hist": chist, "points": F, "picks": picks}
 
 
+def fine_counts_top_down(sizes, C):
+    """Fine clusters per coarse cluster for the top-down hierarchy (NEXT-4).
+
+    The block's C fine clusters are shared out in proportion to the coarse
+    clusters' token counts (largest remainder, ties to the lower coarse
+    cluster), every non-empty coarse cluster getting at least one and at most
+    its token count; empty coarse clusters get none.
+    """
+    sizes = np.asarray(sizes, dtype=np.int64)
+    L = int(sizes.sum())
+    f = np.zeros(sizes.size, dtype=np.int64)
+    if L == 0:
+        return f
+    if int((sizes > 0).sum()) > C:
+        raise ValueError("more non-empty coarse clusters than fine clusters (tokens per coarse centroid < T)")
+    quota = C * sizes / L
+    f = np.where(sizes > 0, np.maximum(1, np.floor(quota).astype(np.int64)), 0)
+    f = np.minimum(f, sizes)
+    rem = quota - np.floor(quota)
+    while f.sum() < C:
+        room = (sizes > 0) & (f < sizes)
+        if not room.any():
+            break
+        cand = np.nonzero(room)[0]
+        c = cand[np.lexsort((cand, -rem[cand]))[0]]    # largest remainder, then lower index
+        f[c] += 1
+        rem[c] = -1.0
+        if (rem[room] < 0).all():
+            rem = np.where(room, quota - np.floor(quota), rem)
+    while f.sum() > C:
+        big = np.nonzero(f > 1)[0]
+        c = big[np.lexsort((big, -f[big]))[0]]          # the largest share, then lower index
+        f[c] -= 1
+    return f
+
+
+def _top_down_block(idx, b, h, j, Xk, Xv, tok0, unit):
+    """Two-level hierarchy for one block, top down (NEXT-4, the other reading
+    of the hierarchical variant): coarse k-means over the block's tokens, then
+    fine k-means inside each coarse cluster, the block's fine clusters shared
+    out by ``fine_counts_top_down``.  Fine slots are laid out by coarse
+    cluster (so each coarse cluster covers a contiguous fine range and token
+    range, as in the bottom-up build); centroids are member means."""
+    cfg, g = idx["cfg"], idx["geom"]
+    dtype, T, Tc = cfg["dtype"], cfg["T"], cfg["Tc"]
+    C_blk, CC_blk = g["C_blk"], g["CC_blk"]
+    L = Xk.shape[0]
+    C = -(-L // T)
+    CC = -(-L // Tc)
+    s0, t0 = j * C_blk, j * CC_blk
+    u = stream_uniforms(cfg["seed"], unit, j, 1, CC)
+    picks = kmeanspp_pick(Xk, CC, u)
+    ca, ccent, chist = lloyd(Xk, Xk[picks], cfg["iters"], dtype)
+    sizes = np.bincount(ca, minlength=CC)
+    f = fine_counts_top_down(sizes, C)
+    Kc = np.zeros((C_blk, Xk.shape[1]))
+    Vc = np.zeros((C_blk, Xk.shape[1]))
+    fine = np.empty(L, dtype=np.int64)                 # block-local fine slot of every token
+    slot = 0
+    coff = np.zeros(CC_blk, dtype=np.int64)
+    for cc in range(CC):
+        coff[cc] = slot
+        if f[cc] == 0:
+            continue
+        members = np.nonzero(ca == cc)[0]              # token order
+        X = Xk[members]
+        # the coarse cluster's own k-means++ stream: the block's level-0 stream key
+        # re-keyed by the coarse index (a generator seeded with seed + cc + 1)
+        uf = stream_uniforms((cfg["seed"] + cc + 1) & _M64, unit, j, 0, int(f[cc]))
+        fp = kmeanspp_pick(X, int(f[cc]), uf)
+        fa, fcent, _ = lloyd(X, X[fp], cfg["iters"], dtype)
+        fine[members] = slot + fa
+        Kc[slot:slot + f[cc]] = fcent
+        Vc[slot:slot + f[cc]] = member_means(Xv[members], fa, int(f[cc]), dtype)
+        slot += int(f[cc])
+    coff[CC:] = slot
+    # the store: tokens by fine slot (slots already grouped by coarse cluster), then token id
+    order = np.argsort(fine, kind="stable")
+    cnt = np.bincount(fine, minlength=C_blk)
+    starts = tok0 + np.concatenate([[0], np.cumsum(cnt)[:-1]])
+    idx["Kc"][b, h, s0:s0 + C_blk] = Kc
+    idx["Vc"][b, h, s0:s0 + C_blk] = Vc
+    idx["off"][b, h, s0:s0 + C_blk] = starts
+    idx["Kp"][b, h, tok0:tok0 + L] = Xk[order]
+    idx["Vp"][b, h, tok0:tok0 + L] = Xv[order]
+    idx["perm"][b, h, tok0:tok0 + L] = tok0 + order
+    idx["assign"][b, h, tok0:tok0 + L] = s0 + fine
+    idx["Kcc"][b, h, t0:t0 + CC_blk] = 0.0
+    idx["Vcc"][b, h, t0:t0 + CC_blk] = 0.0
+    idx["Kcc"][b, h, t0:t0 + CC] = member_means(Xk, ca, CC, dtype, empty=ccent)
+    idx["Vcc"][b, h, t0:t0 + CC] = member_means(Xv, ca, CC, dtype)
+    idx["coff"][b, h, t0:t0 + CC_blk] = s0 + coff
+    return {"coarse_assign": ca, "fine_counts": f, "hist": chist}
+
+
 def _block_init(idx, b, h, j, X, L_old, init_mode, unit, init_given):
     """Initial centroids of one block: k-means++ (R12), given, or warm/stride (R14)."""
     cfg, g = idx["cfg"], idx["geom"]
@@ -389,7 +484,7 @@ def _cluster_block(idx, b, h, j, Xk, Xv, init):
     return hist
 
 
-def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None):
+def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None, hierarchy="bottom_up"):
     """Cluster the first n tokens of every (batch, KV head) from scratch.
 
     K, V: [B, Hkv, >=n, d] arrays whose values are exact in ``cfg['dtype']``.
@@ -397,8 +492,27 @@ def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None):
     ``init_mode``: "kmeans++" (default) or "stride" (slot k of a block starts
     at the key of the block's token k*T).  ``record``: optional dict that
     receives the per-block Lloyd histories keyed by (b, h, j).
+    ``hierarchy`` (two levels only): "bottom_up" (R15: coarse k-means over the
+    fine centroids) or "top_down" (NEXT-4: fine k-means inside each coarse
+    cluster of the block's tokens).
     """
     idx = empty_index(cfg)
+    if hierarchy == "top_down":
+        if cfg.get("levels", 1) != 2 or init is not None or init_mode != "kmeans++":
+            raise ValueError("the top-down hierarchy is a two-level k-means++ build")
+        B, H, Lb = cfg["B"], cfg["Hkv"], cfg["L_blk"]
+        for b in range(B):
+            for h in range(H):
+                for j in range(-(-n // Lb)):
+                    s, e = j * Lb, min(n, (j + 1) * Lb)
+                    rec = _top_down_block(idx, b, h, j, np.asarray(K[b, h, s:e], dtype=np.float64),
+                                          np.asarray(V[b, h, s:e], dtype=np.float64), s, b * H + h)
+                    if record is not None:
+                        record[(b, h, j, "top_down")] = rec
+        idx["n_tokens"] = n
+        idx["n_clustered"] = n
+        _finish_offsets(idx)
+        return idx
     B, H = cfg["B"], cfg["Hkv"]
     Lb = cfg["L_blk"]
     nb = -(-n // Lb)

@@ -589,3 +589,68 @@ def test_per_head_selection_with_the_whole_budget_is_dense_attention():
     idx = mp.build_index(K, V, 200, cfg)
     Q = synth.make_queries(1, 1, 4, cfg["d"], "f32", seed=2)[0]
     np.testing.assert_allclose(mp.decode(idx, Q, 10 ** 6, per_head=True), sdpa(Q, K, V, 200, 2), atol=1e-12)
+
+
+# --------------------------------------------------------------------------- top-down hierarchy (NEXT-4)
+
+def test_fine_counts_share_the_block_by_size():
+    assert list(mp.fine_counts_top_down([100, 0, 30, 5, 1], 34)) == [25, 0, 7, 1, 1]
+    assert list(mp.fine_counts_top_down([10, 10, 10], 4)) == [2, 1, 1]        # remainder ties: lower index
+    assert list(mp.fine_counts_top_down([3, 1], 10)) == [3, 1]               # never more clusters than tokens
+    with pytest.raises(ValueError):
+        mp.fine_counts_top_down([50, 1, 1, 1], 3)                              # a fine cluster for each coarse one
+    f = mp.fine_counts_top_down([7, 9, 0, 40, 8], 16)
+    assert f.sum() == 16 and f[2] == 0 and (f[[0, 1, 3, 4]] >= 1).all()
+
+
+def test_top_down_index_nests_fine_clusters_in_coarse_clusters():
+    """Every coarse cluster owns a contiguous fine-slot range and token range
+    holding exactly its tokens; centroids are member means; the store is a
+    permutation with cluster runs."""
+    cfg = ocfg(B=1, Hkv=2, Hq=4, n_max=256, L_blk=128, T=4, Tc=16, levels=2)
+    K, V, _ = cache(cfg, 256, seed=4)
+    rec = {}
+    idx = mp.build_index(K, V, 256, cfg, hierarchy="top_down", record=rec)
+    g = idx["geom"]
+    for h in range(2):
+        np.testing.assert_array_equal(np.sort(idx["perm"][0, h, :256]), np.arange(256))
+        off, coff = idx["off"][0, h], idx["coff"][0, h]
+        for j in range(2):
+            ca = rec[(0, h, j, "top_down")]["coarse_assign"]
+            for cc in range(g["CC_blk"]):
+                t0, t1 = off[coff[j * g["CC_blk"] + cc]], off[coff[j * g["CC_blk"] + cc + 1]]
+                ids = np.sort(idx["perm"][0, h, t0:t1]) - 128 * j
+                np.testing.assert_array_equal(ids, np.nonzero(ca == cc)[0])
+                if t1 > t0:
+                    np.testing.assert_allclose(idx["Kcc"][0, h, j * g["CC_blk"] + cc],
+                                               K[0, h, 128 * j + ids].astype(np.float64).mean(axis=0), atol=1e-6)
+            for s in range(j * g["C_blk"], (j + 1) * g["C_blk"]):
+                if off[s + 1] > off[s]:
+                    np.testing.assert_allclose(idx["Kc"][0, h, s], idx["Kp"][0, h, off[s]:off[s + 1]].mean(axis=0),
+                                               atol=1e-6)
+                    assert (idx["assign"][0, h, idx["perm"][0, h, off[s]:off[s + 1]]] == s).all()
+
+
+def test_top_down_index_decodes_exactly_when_coarse_clusters_hold_identical_keys():
+    cfg = ocfg(B=1, Hkv=1, Hq=4, n_max=128, L_blk=128, T=4, Tc=32, levels=2)
+    rng = np.random.default_rng(11)
+    protos = rng.standard_normal((4, cfg["d"])).astype(np.float32)
+    K = protos[rng.integers(0, 4, size=128)][None, None]
+    V = rng.standard_normal((1, 1, 128, cfg["d"])).astype(np.float32)
+    idx = mp.build_index(K, V, 128, cfg, hierarchy="top_down")
+    Q = synth.make_queries(1, 1, 4, cfg["d"], "f32", seed=2)[0]
+    for budget, cb in [(1, 1), (8, 40), (30, 128)]:
+        np.testing.assert_allclose(mp.decode(idx, Q, budget, coarse_budget=cb), sdpa(Q, K, V, 128, 1), atol=1e-6)
+
+
+def test_top_down_with_unbounded_budgets_is_dense_and_with_unbounded_coarse_budget_is_flat():
+    cfg = ocfg(B=1, Hkv=2, Hq=4, n_max=256, L_blk=128, T=4, Tc=16, levels=2)
+    K, V, _ = cache(cfg, 256, seed=6)
+    idx = mp.build_index(K, V, 256, cfg, hierarchy="top_down")
+    Q = synth.make_queries(1, 1, 4, cfg["d"], "f32", seed=1)[0]
+    np.testing.assert_allclose(mp.decode(idx, Q, 10 ** 6, coarse_budget=10 ** 6), sdpa(Q, K, V, 256, 2), atol=1e-12)
+    flat = dict(idx)
+    flat["cfg"] = dict(idx["cfg"], levels=1)
+    for budget in [1, 10, 50]:
+        np.testing.assert_allclose(mp.decode(idx, Q, budget, coarse_budget=256), mp.decode(flat, Q, budget),
+                                   atol=1e-12)

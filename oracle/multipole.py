@@ -288,17 +288,28 @@ def _store_block(idx, b, h, j, Xk, Xv, a, cents, tok0):
     idx["assign"][b, h, tok0:tok0 + L] = s0 + a
 
 
+def seq_counts(idx, b):
+    """(n_clustered, n_tokens) of batch element b: the index's counts, or its
+    per-sequence lengths (NEXT-3: a ragged batch, every token clustered)."""
+    if "seq_lens" in idx:
+        nb = int(idx["seq_lens"][b])
+        return nb, nb
+    return idx["n_clustered"], idx["n_tokens"]
+
+
 def _finish_offsets(idx):
-    """Slots of blocks past the clustered range start (and end) at n_clustered."""
+    """Slots of blocks past the clustered range start (and end) at n_clustered
+    (per batch element when the index holds per-sequence lengths)."""
     g = idx["geom"]
-    nc = idx["n_clustered"]
-    nb_used = -(-nc // idx["cfg"]["L_blk"])
-    idx["off"][:, :, nb_used * g["C_blk"]:] = nc
-    if "coff" in idx:
-        # an absent block's fine slots (all empty) form its first coarse range
-        for j in range(nb_used, g["NB"]):
-            idx["coff"][:, :, j * g["CC_blk"]:(j + 1) * g["CC_blk"]] = j * g["C_blk"]
-        idx["coff"][:, :, g["CC_max"]] = g["C_max"]
+    for b in range(idx["cfg"]["B"]):
+        nc = seq_counts(idx, b)[0]
+        nb_used = -(-nc // idx["cfg"]["L_blk"])
+        idx["off"][b, :, nb_used * g["C_blk"]:] = nc
+        if "coff" in idx:
+            # an absent block's fine slots (all empty) form its first coarse range
+            for j in range(nb_used, g["NB"]):
+                idx["coff"][b, :, j * g["CC_blk"]:(j + 1) * g["CC_blk"]] = j * g["C_blk"]
+            idx["coff"][b, :, g["CC_max"]] = g["C_max"]
 
 
 def _coarse_block(idx, b, h, j, L, tok0, unit):
@@ -495,16 +506,27 @@ def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None, hier
     ``hierarchy`` (two levels only): "bottom_up" (R15: coarse k-means over the
     fine centroids) or "top_down" (NEXT-4: fine k-means inside each coarse
     cluster of the block's tokens).
+    ``n`` may be a sequence of B lengths (NEXT-3, a ragged batch): batch
+    element b clusters its first n[b] tokens, blocks aligned to 0 as always,
+    and its decode attends to those tokens only.
     """
     idx = empty_index(cfg)
+    ragged = not np.isscalar(n)
+    if ragged:
+        lens = np.asarray(n, dtype=np.int64)
+        if lens.shape != (cfg["B"],) or (lens < 0).any() or (lens > cfg["n_max"]).any():
+            raise ValueError("per-sequence lengths: B values in [0, n_max]")
+        idx["seq_lens"] = lens
+        n = int(lens.max())
+    n_of = (lambda b: int(idx["seq_lens"][b])) if ragged else (lambda b: n)
     if hierarchy == "top_down":
         if cfg.get("levels", 1) != 2 or init is not None or init_mode != "kmeans++":
             raise ValueError("the top-down hierarchy is a two-level k-means++ build")
         B, H, Lb = cfg["B"], cfg["Hkv"], cfg["L_blk"]
         for b in range(B):
             for h in range(H):
-                for j in range(-(-n // Lb)):
-                    s, e = j * Lb, min(n, (j + 1) * Lb)
+                for j in range(-(-n_of(b) // Lb)):
+                    s, e = j * Lb, min(n_of(b), (j + 1) * Lb)
                     rec = _top_down_block(idx, b, h, j, np.asarray(K[b, h, s:e], dtype=np.float64),
                                           np.asarray(V[b, h, s:e], dtype=np.float64), s, b * H + h)
                     if record is not None:
@@ -515,12 +537,11 @@ def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None, hier
         return idx
     B, H = cfg["B"], cfg["Hkv"]
     Lb = cfg["L_blk"]
-    nb = -(-n // Lb)
     for b in range(B):
         for h in range(H):
             unit = b * H + h
-            for j in range(nb):
-                s, e = j * Lb, min(n, (j + 1) * Lb)
+            for j in range(-(-n_of(b) // Lb)):
+                s, e = j * Lb, min(n_of(b), (j + 1) * Lb)
                 Xk = np.asarray(K[b, h, s:e], dtype=np.float64)
                 Xv = np.asarray(V[b, h, s:e], dtype=np.float64)
                 mode = "kmeans++" if init_mode == "kmeans++" else "stride"
@@ -534,8 +555,8 @@ def build_index(K, V, n, cfg, init=None, init_mode="kmeans++", record=None, hier
     if cfg.get("levels", 1) == 2:
         for b in range(B):
             for h in range(H):
-                for j in range(nb):
-                    s, e = j * Lb, min(n, (j + 1) * Lb)
+                for j in range(-(-n_of(b) // Lb)):
+                    s, e = j * Lb, min(n_of(b), (j + 1) * Lb)
                     ch = _coarse_block(idx, b, h, j, e - s, s, b * H + h)
                     if record is not None:
                         record[(b, h, j, "coarse")] = ch
@@ -648,6 +669,8 @@ def cluster_update(idx, K_new, V_new, record=None):
     receives (b, h, j, keys, init, Lloyd history) per re-clustered block.
     """
     cfg = idx["cfg"]
+    if "seq_lens" in idx:
+        raise ValueError("the update appends the same number of tokens to every sequence: not ragged")
     B, H = cfg["B"], cfg["Hkv"]
     Lb = cfg["L_blk"]
     n0 = idx["n_tokens"]
@@ -756,7 +779,6 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, f
         scale = 1.0 / math.sqrt(d)
     if coarse_budget is None:
         coarse_budget = 8 * budget
-    nc, nt = idx["n_clustered"], idx["n_tokens"]
     if per_head and (cfg.get("levels", 1) != 1 or force_sel is not None):
         raise ValueError("per_head selection is defined for flat indices without forced sets")
     O = np.zeros((B, Hq, d))
@@ -766,6 +788,7 @@ def decode(idx, Q, budget, coarse_budget=None, flags=0, scale=None, info=None, f
             if todo is not None and (b, h) not in todo:
                 continue
             forced = None if force_sel is None else force_sel.get((b, h))
+            nc, nt = seq_counts(idx, b)
             q = np.asarray(Q[b, h * G:(h + 1) * G], dtype=np.float64)
             off = idx["off"][b, h]
             cnt = counts_of(off)

@@ -654,3 +654,50 @@ def test_top_down_with_unbounded_budgets_is_dense_and_with_unbounded_coarse_budg
     for budget in [1, 10, 50]:
         np.testing.assert_allclose(mp.decode(idx, Q, budget, coarse_budget=256), mp.decode(flat, Q, budget),
                                    atol=1e-12)
+
+
+# --------------------------------------------------------------------------- ragged lengths (NEXT-3)
+
+@pytest.mark.parametrize("levels", [1, 2])
+def test_ragged_lengths_equal_to_the_batch_length_are_the_plain_build(levels):
+    cfg = ocfg(B=3, Hkv=2, Hq=4, n_max=256, L_blk=64, T=4, Tc=16, levels=levels)
+    K, V, _ = cache(cfg, 200, seed=9)
+    a = mp.build_index(K, V, 200, cfg)
+    r = mp.build_index(K, V, [200, 200, 200], cfg)
+    for key in ("Kc", "Vc", "off", "Kp", "Vp", "perm", "assign") + (("Kcc", "Vcc", "coff") if levels == 2 else ()):
+        np.testing.assert_array_equal(r[key], a[key])
+    Q = synth.make_queries(1, 3, 4, cfg["d"], "f32", seed=2)[0]
+    np.testing.assert_array_equal(mp.decode(r, Q, 20, coarse_budget=60), mp.decode(a, Q, 20, coarse_budget=60))
+
+
+@pytest.mark.parametrize("levels", [1, 2])
+def test_ragged_batch_attends_each_sequence_to_its_own_tokens(levels):
+    """With every token selected a ragged step is dense attention over each
+    sequence's own first n_b tokens, and tokens past n_b change nothing."""
+    lens = [37, 256, 129, 0]
+    cfg = ocfg(B=4, Hkv=2, Hq=4, n_max=256, L_blk=64, T=4, Tc=16, levels=levels)
+    K, V, _ = cache(cfg, 256, seed=13)
+    idx = mp.build_index(K, V, lens, cfg)
+    Q = synth.make_queries(1, 4, 4, cfg["d"], "f32", seed=5)[0]
+    O = mp.decode(idx, Q, 10 ** 6, coarse_budget=10 ** 6)
+    for b, nb in enumerate(lens):
+        if nb == 0:
+            assert not O[b].any()
+            continue
+        np.testing.assert_allclose(O[b:b + 1], sdpa(Q[b:b + 1], K[b:b + 1], V[b:b + 1], nb, 2), atol=1e-12)
+    K2, V2 = K.copy(), V.copy()
+    for b, nb in enumerate(lens):
+        K2[b, :, nb:] *= -3.0
+        V2[b, :, nb:] += 7.0
+    idx2 = mp.build_index(K2, V2, lens, cfg)
+    for budget in [5, 40]:
+        np.testing.assert_array_equal(mp.decode(idx2, Q, budget, coarse_budget=4 * budget),
+                                      mp.decode(idx, Q, budget, coarse_budget=4 * budget))
+
+
+def test_ragged_index_refuses_the_update():
+    cfg = ocfg(B=2, Hkv=1, Hq=4, n_max=256, L_blk=64, T=4)
+    K, V, _ = cache(cfg, 128, seed=1)
+    idx = mp.build_index(K, V, [100, 128], cfg)
+    with pytest.raises(ValueError):
+        mp.cluster_update(idx, K[:, :, :4], V[:, :, :4])
